@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Benchmark of the HHR decode-time retrieval step on B200.
+
+Workload (default): the Llama-3.1-8B-shaped one-layer decode at 128K context
+(B=1, 32 query / 8 KV heads, d=128, N=131072, 16-token pages, P=512 pages,
+k=4096 tokens, 128-bit codes) on seeded synthetic inputs.
+
+A step is one fused decode call (query prep, page bounds, page top-P,
+Hamming over the kept pages, token top-k, sparse attention) over one
+(sequence batch, layer).  To keep the timed data out of L2 the step cycles
+over `--layers` independent layer instances (distinct K/V/codes/metadata
+buffers, about 50 MiB touched per step, 600 MiB per cycle) captured in one
+CUDA graph.  Key encoding of the full context is timed separately.
+
+`--impl reference` times the CPU oracle (single-threaded C++) on the same
+workload instead, rank 0 only.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import platform
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "µs per HHR decode step at 128K ctx; keys scored/s; % of HBM roofline"
+UNIT = "µs/step"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=48000)
+    ap.add_argument("--warmup", type=int, default=1200)
+    ap.add_argument("--impl", choices=["hhr", "reference"], default="hhr")
+    ap.add_argument("--workload", default="llama8b_128k")
+    ap.add_argument("--layers", type=int, default=12)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def host_info():
+    model = platform.processor() or ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count()
+
+
+def algorithmic_bytes(w, n_valid, P, k):
+    """Bytes a decode step must move at least once (read or write)."""
+    units = w.B * w.Hkv
+    NP = (n_valid + w.page - 1) // w.page
+    Pk = min(P, NP)
+    cand = min(Pk * w.page, n_valid)
+    kk = min(k, cand)
+    parts = dict(
+        meta=units * NP * 2 * w.d * 2,            # bf16 lower/upper bounds of every page
+        codes=units * cand * w.bits // 8,         # codes of the kept pages' tokens
+        kv=units * kk * 2 * w.d * 2,              # gathered K and V rows
+        rw=w.Hkv * (w.d * w.d + w.d * w.bits) * 4,  # R and W (float32)
+        q_out=w.B * w.Hq * w.d * (2 + 4),         # bf16 queries in, float32 out
+        idx=units * (P + k + 1) * 4,              # page_idx, tok_idx, n_sel
+    )
+    return parts, sum(parts.values())
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("decode.cu", "hhr_internal.cuh"):
+        with open(os.path.join(ROOT, "kv_cache_retrieval_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"decode_kernel_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    s = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != kernel_source_hash():
+        return None
+    return int(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except OSError:
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 - 0.05 <= t <= t1 + 0.05]
+        during = bool(rows)
+        if not rows:
+            rows = [s for (_, s) in self.samples]
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                mhz.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz), "during_timed_region": during}
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank number over all ranks (NCCL on GPUs, gloo on CPU)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(us_step_max: float, world: int, keys_per_step: int) -> dict:
+    """Whole-job numbers of a weak-scaling run: every rank decodes its own
+    replica of the workload; the job's step time is the slowest rank's."""
+    return {"value": us_step_max, "keys_scored_per_s": keys_per_step * world / (us_step_max * 1e-6)}
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_hhr(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import kv_cache_retrieval_b200 as hhr
+    from kv_cache_retrieval_b200 import build as kbuild
+    from workloads import get, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if rank == 0:
+        kbuild.build()
+    if world > 1:
+        dist.barrier()
+
+    w = get(args.workload)
+    inp = make_inputs(w)
+    n_valid = w.N
+    L = max(1, args.layers)
+    dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap)
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    K0, V0 = bf(inp.K), bf(inp.V)
+    q_host = torch.from_numpy(np.ascontiguousarray(inp.q[0]).view(np.int16)).view(torch.bfloat16)
+    q_dev = q_host.to(dev)
+    R = torch.from_numpy(inp.R).to(dev)
+    W = torch.from_numpy(inp.W).to(dev)
+    codes0 = torch.zeros(w.B, w.Hkv, w.n_cap, w.words, dtype=torch.int32, device=dev)
+    meta0 = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=torch.bfloat16, device=dev)
+
+    # key encoding of the whole context, timed separately
+    s = torch.cuda.current_stream()
+    for _ in range(2):
+        hhr.hhr_encode_keys(dims, K0, R, W, 0, n_valid, codes0, meta0)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    e0.record(s)
+    for _ in range(reps):
+        hhr.hhr_encode_keys(dims, K0, R, W, 0, n_valid, codes0, meta0)
+    e1.record(s)
+    torch.cuda.synchronize()
+    enc_ms = e0.elapsed_time(e1) / reps
+    enc_flops = 2.0 * w.B * w.Hkv * n_valid * w.d * (w.d + w.bits)
+
+    layers = []
+    for li in range(L):
+        lay = dict(
+            K=K0 if li == 0 else K0.clone(), V=V0 if li == 0 else V0.clone(),
+            codes=codes0 if li == 0 else codes0.clone(), meta=meta0 if li == 0 else meta0.clone(),
+            q=q_dev.clone(),
+            page_idx=torch.empty(w.B, w.Hkv, w.P, dtype=torch.int32, device=dev),
+            tok_idx=torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=dev),
+            n_sel=torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev),
+            out=torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev))
+        layers.append(lay)
+    ws = torch.zeros(hhr.hhr_workspace_size(dims, w.P, w.k), dtype=torch.uint8, device=dev)
+    scale = 1.0 / math.sqrt(w.d)
+
+    def step(lay, stream=None):
+        hhr.hhr_decode_step(dims, lay["q"], R, W, lay["codes"], lay["meta"], lay["K"], lay["V"],
+                            n_valid, w.P, w.k, scale, lay["page_idx"], lay["tok_idx"], lay["n_sel"],
+                            lay["out"], ws, None, stream)
+
+    # warm-up (eager), then one CUDA graph per cycle over the layer instances
+    for i in range(max(3, args.warmup)):
+        step(layers[i % L])
+    torch.cuda.synchronize()
+    assert hhr.hhr_read_status(ws) == hhr.HHR_OK
+
+    K = max(1, args.steps)
+    launch = "cuda-graph"
+    graphs = {}
+    try:
+        cap_stream = torch.cuda.Stream()
+        for n in sorted({L, K % L} - {0}):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="relaxed"):
+                for li in range(n):
+                    step(layers[li], cap_stream.cuda_stream)
+            graphs[n] = g
+        for g in graphs.values():
+            g.replay()
+        torch.cuda.synchronize()
+    except Exception as exc:  # capture unsupported: time eager launches instead
+        launch = f"stream (graph capture failed: {type(exc).__name__})"
+        graphs = {}
+        torch.cuda.synchronize()
+
+    gpu_uuid = f"GPU-{torch.cuda.get_device_properties(dev).uuid}"
+    sampler = ClockSampler(gpu_uuid)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    t0 = time.time()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(s)
+    if graphs:
+        for _ in range(K // L):
+            graphs[L].replay()
+        if K % L:
+            graphs[K % L].replay()
+    else:
+        for i in range(K):
+            step(layers[i % L])
+    ev1.record(s)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    status = hhr.hhr_read_status(ws)
+    assert status == hhr.HHR_OK, hhr.hhr_status_string(status)
+
+    us_step = ms * 1000.0 / K
+    keys_per_step = w.B * w.Hkv * n_valid
+    agg = aggregate(us_step, world, keys_per_step)
+    parts, alg = algorithmic_bytes(w, n_valid, w.P, w.k)
+    peak, peak_kind = measured_peak()
+    achieved = alg / (us_step * 1e-6) / 1e9
+
+    # end to end through the public API: pinned q in, decode, out back
+    q_pin = q_host.pin_memory()
+    out_pin = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32).pin_memory()
+    lay0 = layers[0]
+    n_e2e = max(1, min(args.e2e_steps, K))
+    for _ in range(20):
+        lay0["q"].copy_(q_pin, non_blocking=True)
+        step(lay0)
+        out_pin.copy_(lay0["out"], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    if world > 1:
+        dist.barrier()
+    te0 = time.perf_counter()
+    for i in range(n_e2e):
+        lay = layers[i % L]
+        lay["q"].copy_(q_pin, non_blocking=True)
+        step(lay)
+        out_pin.copy_(lay["out"], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    te1 = time.perf_counter()
+    e2e_us = max_over_ranks((te1 - te0) * 1e6 / n_e2e, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, w, n_valid, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(agg["value"], 3), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": us_step / 1000.0,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; Llama-3.1-8B-shaped keys/values/queries, planted keys)",
+            "config": {
+                "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": n_valid,
+                "page": w.page, "P": w.P, "k": w.k, "bits": w.bits, "global_batch": w.B * world,
+                "seq_len": n_valid, "parallelism": f"replicas x{world} (independent units)",
+                "layers_cycled": L, "l2": f"inputs larger than L2: {L} layer instances cycled "
+                f"({alg * L / 2**20:.0f} MiB touched per cycle)", "launch": launch,
+            },
+            "keys_scored_per_s": agg["keys_scored_per_s"],
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": profiled_traffic(w.name), "peak_source": peak_kind,
+                         "algorithmic_bytes": alg, "bytes_breakdown": parts,
+                         "kernel": "decode_kernel<4,4,fused>"},
+            "e2e": {"value": round(e2e_us, 3), "unit": UNIT,
+                    "h2d_bytes_per_step": int(q_pin.numel() * q_pin.element_size()),
+                    "d2h_bytes_per_step": int(out_pin.numel() * out_pin.element_size()),
+                    "steps": n_e2e, "how": "pinned q H2D + hhr_decode_step + out D2H + sync, per step"},
+            "gpu_launches": K,
+            "clocks": clocks,
+            "encode": {"ms": round(enc_ms, 4), "keys": w.B * w.Hkv * n_valid,
+                       "tflops_useful": round(enc_flops / (enc_ms * 1e-3) / 1e12, 2)},
+            "cpu_baseline": cpu,
+            "context": "pages' own numbers (A800, PyTorch): 3.30x decode and 2.83x end-to-end "
+                       "speedup over dense attention at 128K, Llama-3.1-8B-Instruct",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        graphs.clear()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------- oracle (CPU)
+
+def _oracle_unit_sample(inp, w, n_valid):
+    """Oracle state for unit (0, 0): encoded keys (not timed)."""
+    from oracle import oracle as O
+    import numpy as np
+    codes = np.zeros((w.B, w.Hkv, w.n_cap, w.words), np.uint32)
+    meta = np.zeros((w.B, w.Hkv, w.np_cap, 2, w.d), np.uint16)
+    O.encode_all(inp, 0, n_valid, codes=codes, meta=meta, units=[(0, 0)])
+    return codes, meta
+
+
+def _oracle_step(inp, w, codes, meta, n_valid):
+    from oracle import oracle as O
+    r = w.r
+    O.decode_unit(inp.q[0, 0, 0:r], inp.R[0], inp.W[0], codes[0, 0], meta[0, 0], inp.K[0, 0],
+                  inp.V[0, 0], n_valid, w.page, w.P, w.k, 1.0 / math.sqrt(w.d))
+
+
+def cpu_baseline(inp, w, n_valid, seconds):
+    codes, meta = _oracle_unit_sample(inp, w, n_valid)
+    units = w.B * w.Hkv
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        _oracle_step(inp, w, codes, meta, n_valid)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    per_unit = (time.perf_counter() - t0) / n
+    model, ncpu = host_info()
+    return {"value": round(per_unit * units * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"oracle decode of unit (0,0) of {units}, {n} runs in {seconds:.0f}s, "
+                      f"scaled by {units}", "host_cpu": model, "host_nproc": ncpu}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from workloads import get, make_inputs
+    w = get(args.workload)
+    inp = make_inputs(w)
+    n_valid = w.N
+    codes, meta = _oracle_unit_sample(inp, w, n_valid)
+    units = w.B * w.Hkv
+    for _ in range(max(1, min(args.warmup, 3))):
+        _oracle_step(inp, w, codes, meta, n_valid)
+    budget = 150.0
+    t0 = time.perf_counter()
+    n = 0
+    while n < args.steps:
+        _oracle_step(inp, w, codes, meta, n_valid)
+        n += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    per_step_us = (time.perf_counter() - t0) / n * units * 1e6
+    model, ncpu = host_info()
+    sample = (f"each step: oracle decode of unit (0,0) of {units} (scaled by {units}); "
+              f"{n} of {args.steps} requested steps timed within {budget:.0f}s")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(per_step_us, 1), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "steps_timed": n, "warmup": args.warmup,
+        "ms_per_step": per_step_us / 1000.0, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": n_valid,
+                   "page": w.page, "P": w.P, "k": w.k, "bits": w.bits},
+        "cpu_baseline": {"value": round(per_step_us, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample, "host_cpu": model, "host_nproc": ncpu},
+        "e2e": {"value": round(per_step_us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_hhr(args)
+
+
+if __name__ == "__main__":
+    main()

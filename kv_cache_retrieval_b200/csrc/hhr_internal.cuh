@@ -1,0 +1,136 @@
+// Internal declarations shared by the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "hhr.h"
+
+namespace hhr {
+
+constexpr int kD = 128;                 // head dimension handled by every kernel
+constexpr int kDecodeThreads = 512;     // one decode CTA per SM, 16 warps
+constexpr int kMaxCtasPerUnit = 64;     // CTAs that may share one (sequence, KV head)
+constexpr int kMinPagesPerCta = 32;     // below this a unit uses fewer CTAs
+constexpr int kBuckets = 2048;          // page top-P histogram bins
+constexpr int kCandMax = 1024;          // boundary-bucket candidates ranked exactly
+constexpr int kMaxTokensPerCta = 16384; // candidate tokens one CTA scores
+constexpr int kAttnChunk = 32;          // tokens per K/V staging stage
+constexpr int kAttnStages = 4;          // depth of the K/V staging ring
+constexpr unsigned long long kSpinLimit = 1ull << 31;  // ~1 s at 2 GHz
+
+inline __host__ __device__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout (bytes).  The status word sits at offset 0.
+struct WsLayout {
+  size_t status, counters, U, minmax, hist, part, total;
+  int np_stride;  // floats per unit in the U area (multiple of 4)
+};
+
+inline __host__ __device__ WsLayout ws_layout(int units, int np_cap, int r, int bits) {
+  WsLayout L;
+  size_t off = 0;
+  L.status = off;   off += 256;
+  L.counters = off; off += align_up(sizeof(uint32_t) * (size_t)units, 256);
+  L.np_stride = (int)align_up((size_t)np_cap, 4);
+  L.U = off;        off += align_up(sizeof(float) * (size_t)units * L.np_stride, 256);
+  L.minmax = off;   off += align_up(sizeof(float) * 2 * (size_t)units * kMaxCtasPerUnit, 256);
+  L.hist = off;     off += align_up(sizeof(int32_t) * (size_t)units * kMaxCtasPerUnit * (bits + 1), 256);
+  L.part = off;     off += align_up(sizeof(float) * (size_t)units * kMaxCtasPerUnit * r * (kD + 2), 256);
+  L.total = off;
+  return L;
+}
+
+enum DecodeMode : int { kModeSelect = 0, kModeFused = 1, kModeAttend = 2 };
+
+struct DecodeArgs {
+  // inputs
+  const uint16_t* q;        // bf16 [B][Hq][d]
+  const float* R;           // [Hkv][d][d]
+  const float* W;           // [Hkv][d][bits]
+  const uint32_t* codes;    // [B][Hkv][n_cap][w]
+  const uint16_t* meta;     // bf16 [B][Hkv][np_cap][2][d]
+  const uint16_t* K;        // bf16 [B][Hkv][n_cap][d]
+  const uint16_t* V;
+  const int32_t* tok_in;    // attend-only: [B][Hkv][k]
+  const int32_t* nsel_in;   // attend-only: [B][Hkv]
+  // outputs
+  int32_t* page_idx;        // [B][Hkv][P]
+  int32_t* tok_idx;         // [B][Hkv][k]
+  int32_t* n_sel;           // [B][Hkv]
+  float* out;               // [B][Hq][d]
+  float* dbg_U;             // nullable [B][Hkv][NP]
+  int32_t* dbg_D;           // nullable [B][Hkv][P*page]
+  // workspace
+  uint32_t* status;
+  uint32_t* counters;
+  float* wsU;
+  float* wsMinMax;
+  int32_t* wsHist;
+  float* wsPart;
+  int np_stride;
+  // sizes
+  int B, Hq, Hkv, units, page, n_cap, np_cap, n_valid, NP, P, Pk, k, C, grid_units;
+  int slice_pages;          // max kept pages one CTA scores (ceil(Pk / C))
+  int slice_tokens;         // max tokens one CTA scores or attends
+  float scale_log2;         // scale * log2(e)
+  unsigned long long spin_limit;
+};
+
+struct EncodeArgs {
+  const uint16_t* K;
+  const float* R;
+  const float* W;
+  uint32_t* codes;
+  uint16_t* meta;
+  int Hkv, units, bits, page, n_cap, np_cap, n_begin, n_end, tile_begin, n_tiles;
+};
+
+// Shared-memory bytes of a decode CTA (host and device agree on the carve-up).
+struct DecodeSmem {
+  size_t qt, qf, qc, my_pages, tokD, sel, scratch, total;
+};
+
+inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, int r, int mode) {
+  size_t sel = 0, hist = 0, attn = 0;
+  if (mode != kModeAttend) {
+    sel = sizeof(float) * align_up((size_t)NP, 4)          // U of every page
+        + sizeof(int) * kBuckets                             // histogram
+        + sizeof(uint32_t) * align_up(((size_t)NP + 31) / 32, 4)  // kept bitmap
+        + (sizeof(float) + sizeof(int)) * kCandMax;          // boundary candidates
+    hist = sizeof(int) * (size_t)C * (bits + 1) + 16;
+  }
+  if (mode != kModeSelect) {
+    const size_t ring = (size_t)kAttnStages * kAttnChunk * 2 * kD * sizeof(uint16_t);
+    const size_t merge = sizeof(float) * (kDecodeThreads / 32) * (size_t)r * (kD + 2);
+    attn = ring > merge ? ring : merge;
+  }
+  size_t m = sel > hist ? sel : hist;
+  return m > attn ? m : attn;
+}
+
+inline __host__ __device__ DecodeSmem decode_smem(int NP, int C, int bits, int r, int slice_pages,
+                                                  int slice_tokens, int mode) {
+  DecodeSmem s;
+  size_t off = 0;
+  s.qt = off;       off += align_up(sizeof(float) * r * kD, 16);
+  s.qf = off;       off += align_up(sizeof(float) * r * kD, 16);
+  s.qc = off;       off += align_up(sizeof(uint32_t) * r * (bits / 32), 16);
+  s.my_pages = off; off += align_up(sizeof(int) * (size_t)(slice_pages + 1), 16);
+  s.tokD = off;     off += align_up(sizeof(uint16_t) * (size_t)(slice_tokens + 1), 16);
+  s.sel = off;      off += align_up(sizeof(int) * (size_t)(slice_tokens + 1), 16);
+  s.scratch = off;  off += align_up(decode_scratch_bytes(NP, C, bits, r, mode), 16);
+  s.total = off;
+  return s;
+}
+
+// Launchers (defined in decode.cu / encode.cu).  Return a cudaError_t.
+cudaError_t launch_decode(const DecodeArgs& a, int r, int bits, int mode, size_t smem_bytes,
+                          cudaStream_t stream);
+cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t stream);
+cudaError_t launch_wait_timeout(uint32_t* status, uint32_t* counter, unsigned long long spin,
+                                cudaStream_t stream);
+
+}  // namespace hhr

@@ -1,0 +1,191 @@
+"""Helpers shared by the GPU parity tests: move seeded inputs to the device,
+run the CUDA path through the C ABI, and compare with the oracle under the
+parity rules:
+
+* codes and Hamming distances bit-exact, except projections whose oracle
+  value has |z| < 1e-4 (counted and reported);
+* page and token index sets identical, except candidates whose score lies
+  within 1e-3 (relative) of the cutoff score (reported);
+* attention outputs within 2e-3 max-abs.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import kv_cache_retrieval_b200 as hhr
+from oracle import oracle as O
+from workloads import bf16_bits_to_f32
+
+ATTN_TOL = 2e-3
+NEAR_CUTOFF = 1e-3
+
+
+def bf16_dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def u32_dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).cuda()
+
+
+def bits_host(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def u32_host(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint32)
+
+
+class Dev:
+    """Device copies of a workload's inputs plus output buffers."""
+
+    def __init__(self, inp, P=None, k=None):
+        w = inp.w
+        self.w = w
+        self.inp = inp
+        self.P = w.P if P is None else P
+        self.k = w.k if k is None else k
+        self.dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap)
+        self.K = bf16_dev(inp.K)
+        self.V = bf16_dev(inp.V)
+        self.q = bf16_dev(inp.q)                   # [steps][B][Hq][d]
+        self.R = torch.from_numpy(inp.R).cuda()
+        self.W = torch.from_numpy(inp.W).cuda()
+        self.codes = torch.zeros(w.B, w.Hkv, w.n_cap, w.words, dtype=torch.int32, device="cuda")
+        self.meta = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=torch.bfloat16, device="cuda")
+        self.page_idx = torch.full((w.B, w.Hkv, self.P), -7, dtype=torch.int32, device="cuda")
+        self.tok_idx = torch.full((w.B, w.Hkv, self.k), -7, dtype=torch.int32, device="cuda")
+        self.n_sel = torch.full((w.B, w.Hkv), -7, dtype=torch.int32, device="cuda")
+        self.out = torch.full((w.B, w.Hq, w.d), float("nan"), dtype=torch.float32, device="cuda")
+        ws = hhr.hhr_workspace_size(self.dims, self.P, self.k)
+        self.ws = torch.zeros(ws, dtype=torch.uint8, device="cuda")
+        self.scale = 1.0 / math.sqrt(w.d)
+
+    def encode(self, n_begin=0, n_end=None):
+        n_end = self.w.N if n_end is None else n_end
+        hhr.hhr_encode_keys(self.dims, self.K, self.R, self.W, n_begin, n_end, self.codes, self.meta)
+
+    def load_state(self, codes: np.ndarray, meta: np.ndarray):
+        """Use oracle-encoded codes / metadata (identical bytes) as the state."""
+        self.codes.copy_(u32_dev(codes))
+        self.meta.copy_(bf16_dev(meta))
+
+    def select(self, step=0, n_valid=None, dbg=True):
+        w = self.w
+        n_valid = self.inp.n_valid(step) if n_valid is None else n_valid
+        NP = (n_valid + w.page - 1) // w.page
+        self.dbg_U = torch.full((w.B, w.Hkv, max(NP, 1)), float("nan"), device="cuda") if dbg else None
+        self.dbg_D = torch.full((w.B, w.Hkv, self.P * w.page), -7, dtype=torch.int32, device="cuda") if dbg else None
+        hhr.hhr_select(self.dims, self.q[step], self.R, self.W, self.codes, self.meta, n_valid, self.P,
+                       self.k, self.page_idx, self.tok_idx, self.n_sel, self.dbg_U, self.dbg_D, self.ws)
+
+    def attend(self, step, tok_idx, n_sel):
+        hhr.hhr_sparse_attend(self.dims, self.q[step], self.K, self.V, tok_idx, n_sel, self.k,
+                              self.scale, self.out, self.ws)
+
+    def decode(self, step=0, n_valid=None):
+        n_valid = self.inp.n_valid(step) if n_valid is None else n_valid
+        hhr.hhr_decode_step(self.dims, self.q[step], self.R, self.W, self.codes, self.meta, self.K,
+                            self.V, n_valid, self.P, self.k, self.scale, self.page_idx, self.tok_idx,
+                            self.n_sel, self.out, self.ws)
+
+    def status(self):
+        return hhr.hhr_read_status(self.ws)
+
+
+# ----------------------------------------------------------------- comparisons
+
+def compare_encode(inp, codes_g, meta_g, units, n_end, n_begin=0):
+    """Codes bit-exact except oracle |z| < 1e-4; metadata equal (a differing
+    bound may only be one bf16 step further out or in, reported)."""
+    w = inp.w
+    report = dict(code_bits=0, ambiguous=0, meta_vals=0, meta_diff=0)
+    codes_o, meta_o, _ = O.encode_all(inp, n_begin=0, n_end=n_end, units=units)
+    for (b, g) in units:
+        c_o, _, z = O.project_sign(inp.K[b, g, n_begin:n_end], inp.W[g], want_z=True)
+        c_g = codes_g[b, g, n_begin:n_end]
+        bits_o = np.unpackbits(c_o.view(np.uint8), bitorder="little").reshape(z.shape)
+        bits_g = np.unpackbits(np.ascontiguousarray(c_g).view(np.uint8), bitorder="little").reshape(z.shape)
+        amb = np.abs(z) < 1e-4
+        bad = (bits_o != bits_g) & ~amb
+        assert not bad.any(), f"unit {(b, g)}: {int(bad.sum())} code bits differ with |z| >= 1e-4"
+        report["code_bits"] += bits_o.size
+        report["ambiguous"] += int(amb.sum())
+        p0, p1 = n_begin // w.page, (n_end + w.page - 1) // w.page
+        mo = meta_o[b, g, p0:p1].astype(np.int32)
+        mg = meta_g[b, g, p0:p1].astype(np.int32)
+        diff = mo != mg
+        report["meta_vals"] += mo.size
+        report["meta_diff"] += int(diff.sum())
+        if diff.any():
+            # The GPU rotates in float32, the oracle in double.  A stored
+            # bound may differ by the float32 dot-product error bound
+            # (gamma_128 * sum_i |k_i R_ij| <= 1e-5 * sum_i |k_i R_ij|) plus
+            # one bf16 step at the larger of the two values.
+            t0 = p0 * w.page
+            kf = np.abs(bf16_bits_to_f32(inp.K[b, g, t0:n_end]).astype(np.float64))
+            mag = kf @ np.abs(inp.R[g].astype(np.float64))              # [n][d]
+            pad = (p1 - p0) * w.page - mag.shape[0]
+            mag = np.pad(mag, ((0, pad), (0, 0))).reshape(p1 - p0, w.page, w.d).max(1)
+            eps = np.broadcast_to((1e-5 * mag)[:, None, :], mo.shape)
+            fo = bf16_bits_to_f32(meta_o[b, g, p0:p1]).astype(np.float64)
+            fg = bf16_bits_to_f32(meta_g[b, g, p0:p1]).astype(np.float64)
+            step = np.maximum(np.abs(fo), np.abs(fg)) * 2.0 ** -7
+            ok = np.abs(fo - fg) <= eps + step + 1e-30
+            assert np.all(ok[diff]), "metadata differs by more than the float32 rotation error"
+    return report
+
+
+def compare_select(w, ores, page_idx, tok_idx, n_sel, units, dbg_U=None, dbg_D=None, P=None,
+                   k=None):
+    """Compare one decode step's selection for the given units."""
+    P = w.P if P is None else P
+    k = w.k if k is None else k
+    rep = dict(units=0, near_cutoff_pages=0, page_set_diff=0, tok_set_diff=0, q_ambiguous=0)
+    for (b, g) in units:
+        rep["units"] += 1
+        U_o = ores["U"][(b, g)]
+        NP = U_o.shape[0]
+        po = ores["page_idx"][b, g]
+        pg = page_idx[b, g]
+        if dbg_U is not None and NP:
+            ug = dbg_U[b, g, :NP].astype(np.float64)
+            tol = 2e-5 * (np.abs(U_o) + np.abs(U_o).mean() + 1.0)
+            assert np.all(np.abs(ug - U_o) <= tol), f"unit {(b, g)}: page bounds differ"
+        so, sg = set(po[po >= 0].tolist()), set(pg[pg >= 0].tolist())
+        assert len(sg) == len(so) == min(P, NP)
+        assert np.all(pg[len(sg):] == -1) and np.all(np.diff(pg[:len(sg)]) > 0)
+        if so != sg:
+            cut = np.sort(U_o)[::-1][min(P, NP) - 1]
+            for p in so ^ sg:
+                assert abs(U_o[p] - cut) <= NEAR_CUTOFF * max(abs(cut), 1e-30), \
+                    f"unit {(b, g)}: page {p} differs but is not near the cutoff"
+            rep["page_set_diff"] += 1
+            rep["near_cutoff_pages"] += len(so ^ sg)
+        qa = int(ores["q_ambiguous"][b, g])
+        rep["q_ambiguous"] += qa
+        to, tg = ores["tok_idx"][b, g], tok_idx[b, g]
+        ns = int(ores["n_sel"][b, g])
+        if so == sg and qa == 0:
+            assert int(n_sel[b, g]) == ns
+            assert np.array_equal(to, tg), f"unit {(b, g)}: token selection differs"
+            if dbg_D is not None:
+                assert np.array_equal(ores["D"][b, g], dbg_D[b, g]), f"unit {(b, g)}: distances differ"
+        else:
+            # a near-cutoff page swap or an ambiguous query bit changes the
+            # candidate set; the token sets are then reported, not compared
+            rep["tok_set_diff"] += int(len(set(to[to >= 0].tolist()) ^ set(tg[tg >= 0].tolist())))
+    return rep
+
+
+def compare_out(w, out_o, out_g, units):
+    r = w.r
+    err = 0.0
+    for (b, g) in units:
+        e = float(np.abs(out_o[b, g * r:(g + 1) * r] - out_g[b, g * r:(g + 1) * r]).max())
+        err = max(err, e)
+    assert err <= ATTN_TOL, f"attention max-abs error {err}"
+    return err

@@ -1,0 +1,267 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Small cases span several CTAs per unit and ragged
+tails; the full-size workloads run in the benchmark's launch configuration
+and are checked on sampled (sequence, KV head) units."""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_retrieval_b200 as hhr
+from gpu_harness import (Dev, bits_host, compare_encode, compare_out, compare_select, u32_host)
+from oracle import oracle as O
+from workloads import get, make_inputs, scaled
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny_4k": get("tiny_4k"),
+    "llama_20k_ragged": scaled(get("llama8b_32k"), N=20003),
+    "b256_s32": scaled(get("batch8_64k_b256"), B=2, N=9001, P=64, k=1024),
+    "rope_appends": scaled(get("qwen8b_128k_rope"), B=2, N=7000, P=64, k=512, appends=4),
+    "page1": scaled(get("llama8b_32k"), Hq=8, Hkv=2, N=700, page=1, P=100, k=50, planted=4),
+    "page64": scaled(get("llama8b_32k"), Hq=8, Hkv=2, N=5000, page=64, P=20, k=300, planted=4),
+    "gqa2": scaled(get("llama8b_32k"), Hq=16, Hkv=8, N=3000, P=40, k=200, planted=8),
+    "gqa8": scaled(get("llama8b_32k"), Hq=32, Hkv=4, N=3000, P=40, k=200, planted=8),
+}
+
+_cache = {}
+
+
+def case(name):
+    if name not in _cache:
+        w = SMALL[name]
+        inp = make_inputs(w)
+        codes, meta, _ = O.encode_all(inp, n_end=w.N)
+        _cache[name] = (inp, codes, meta)
+    return _cache[name]
+
+
+def all_units(w):
+    return [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_encode_matches_oracle(name):
+    inp, _, _ = case(name)
+    w = inp.w
+    d = Dev(inp)
+    d.encode(0, w.N)
+    torch.cuda.synchronize()
+    rep = compare_encode(inp, u32_host(d.codes), bits_host(d.meta), all_units(w), w.N)
+    print(name, rep)
+
+
+def test_append_encoding_matches_oracle():
+    inp, _, _ = case("llama_20k_ragged")
+    w = inp.w
+    d = Dev(inp)
+    n = w.N
+    d.encode(0, n - 9)
+    for a, b in [(n - 9, n - 8), (n - 8, n - 5), (n - 5, n - 4), (n - 4, n)]:
+        d.encode(a, b)
+    torch.cuda.synchronize()
+    compare_encode(inp, u32_host(d.codes), bits_host(d.meta), all_units(w), n)
+
+
+def _host(t):
+    return t.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_select_matches_oracle(name):
+    inp, codes, meta = case(name)
+    w = inp.w
+    step = inp.steps - 1
+    ores = O.decode_all(inp, codes, meta, step=step, attend_too=False)
+    d = Dev(inp)
+    d.load_state(codes, meta)
+    d.select(step=step)
+    assert d.status() == hhr.HHR_OK
+    rep = compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), all_units(w),
+                         dbg_U=_host(d.dbg_U), dbg_D=_host(d.dbg_D))
+    print(name, rep)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attend_matches_oracle_on_oracle_indices(name):
+    inp, codes, meta = case(name)
+    w = inp.w
+    ores = O.decode_all(inp, codes, meta)
+    d = Dev(inp)
+    tok = torch.from_numpy(ores["tok_idx"]).cuda()
+    nsel = torch.from_numpy(ores["n_sel"]).cuda()
+    d.attend(0, tok, nsel)
+    assert d.status() == hhr.HHR_OK
+    err = compare_out(w, ores["out"], _host(d.out), all_units(w))
+    print(name, "max abs err", err)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_fused_decode_matches_oracle(name):
+    inp, codes, meta = case(name)
+    w = inp.w
+    ores = O.decode_all(inp, codes, meta)
+    d = Dev(inp)
+    d.load_state(codes, meta)
+    d.decode(0)
+    assert d.status() == hhr.HHR_OK
+    rep = compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), all_units(w))
+    if rep["page_set_diff"] == 0 and rep["q_ambiguous"] == 0:
+        compare_out(w, ores["out"], _host(d.out), all_units(w))
+    print(name, rep)
+
+
+@pytest.mark.parametrize("name", ["tiny_4k", "llama_20k_ragged", "b256_s32"])
+def test_gpu_encode_then_decode_matches_oracle(name):
+    inp, codes, meta = case(name)
+    w = inp.w
+    ores = O.decode_all(inp, codes, meta)
+    d = Dev(inp)
+    d.encode(0, w.N)
+    d.decode(0)
+    assert d.status() == hhr.HHR_OK
+    rep = compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), all_units(w))
+    if rep["page_set_diff"] == 0 and rep["q_ambiguous"] == 0:
+        compare_out(w, ores["out"], _host(d.out), all_units(w))
+    print(name, rep)
+
+
+def test_rope_appends_each_step():
+    """Encode the context, then per decode step append one key and decode."""
+    inp, _, _ = case("rope_appends")
+    w = inp.w
+    d = Dev(inp)
+    d.encode(0, w.N)
+    codes = np.zeros((w.B, w.Hkv, w.n_cap, w.words), np.uint32)
+    meta = np.zeros((w.B, w.Hkv, w.np_cap, 2, w.d), np.uint16)
+    O.encode_all(inp, 0, w.N, codes=codes, meta=meta)
+    for step in range(w.appends):
+        d.encode(w.N + step, w.N + step + 1)
+        O.encode_all(inp, w.N + step, w.N + step + 1, codes=codes, meta=meta)
+        d.decode(step)
+        ores = O.decode_all(inp, codes, meta, step=step)
+        rep = compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), all_units(w))
+        if rep["page_set_diff"] == 0 and rep["q_ambiguous"] == 0:
+            compare_out(w, ores["out"], _host(d.out), all_units(w))
+    torch.cuda.synchronize()
+    compare_encode(inp, u32_host(d.codes), bits_host(d.meta), all_units(w), w.n_cap)
+    assert d.status() == hhr.HHR_OK
+
+
+# ------------------------------------------------------------------ edge cases
+
+@pytest.mark.parametrize("n_valid", [0, 1, 5, 16, 17, 333, 4096])
+def test_edge_context_lengths(n_valid):
+    inp, codes, meta = case("tiny_4k")
+    w = inp.w
+    d = Dev(inp)
+    d.load_state(codes, meta)
+    # oracle on the (possibly truncated) context of the single unit
+    res = O.decode_unit(inp.q[0, 0, 0:1], inp.R[0], inp.W[0], codes[0, 0], meta[0, 0],
+                        inp.K[0, 0], inp.V[0, 0], n_valid, w.page, w.P, w.k, d.scale)
+    ores = dict(page_idx=res["page_idx"][None, None], tok_idx=res["tok_idx"][None, None],
+                n_sel=np.array([[res["n_sel"]]]), out=res["out"][None],
+                D=res["D"][None, None], q_ambiguous=np.array([[res["q_ambiguous"]]]),
+                U={(0, 0): res["U"]})
+    d.decode(0, n_valid=n_valid)
+    assert d.status() == hhr.HHR_OK
+    compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), [(0, 0)])
+    compare_out(w, ores["out"], _host(d.out), [(0, 0)])
+    d.select(0, n_valid=n_valid)
+    compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), [(0, 0)],
+                   dbg_U=_host(d.dbg_U), dbg_D=_host(d.dbg_D))
+
+
+@pytest.mark.parametrize("P,k", [(10_000, 128), (32, 100_000), (10_000, 100_000), (1, 1)])
+def test_budget_extremes(P, k):
+    inp, codes, meta = case("llama_20k_ragged")
+    w = inp.w
+    ores = O.decode_all(inp, codes, meta, P=P, k=k)
+    d = Dev(inp, P=P, k=k)
+    d.load_state(codes, meta)
+    d.decode(0)
+    assert d.status() == hhr.HHR_OK
+    rep = compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), all_units(w),
+                         P=P, k=k)
+    if rep["page_set_diff"] == 0 and rep["q_ambiguous"] == 0:
+        compare_out(w, ores["out"], _host(d.out), all_units(w))
+
+
+def test_degenerate_all_equal_scores():
+    """Zero keys: every page bound is equal and every code is zero, so the
+    selection is decided by the index tie-breaks alone."""
+    w = scaled(get("llama8b_32k"), Hq=8, Hkv=2, N=3000, P=50, k=300, planted=0)
+    inp = make_inputs(w)
+    inp.K[:] = 0
+    codes, meta, _ = O.encode_all(inp)
+    ores = O.decode_all(inp, codes, meta)
+    d = Dev(inp)
+    d.encode(0, w.N)
+    d.decode(0)
+    assert d.status() == hhr.HHR_OK
+    compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), all_units(w))
+    compare_out(w, ores["out"], _host(d.out), all_units(w))
+    assert _host(d.page_idx)[0, 0].tolist() == list(range(50))
+
+
+def test_workspace_is_reusable_and_results_repeat():
+    inp, codes, meta = case("llama_20k_ragged")
+    d = Dev(inp)
+    d.load_state(codes, meta)
+    outs = []
+    for _ in range(3):
+        d.decode(0)
+        outs.append((_host(d.tok_idx).copy(), _host(d.out).copy()))
+    assert d.status() == hhr.HHR_OK
+    for t, o in outs[1:]:
+        assert np.array_equal(t, outs[0][0]) and np.array_equal(o, outs[0][1])
+    # the per-unit counters (4 bytes each, at offset 256) are back to zero
+    units = inp.w.B * inp.w.Hkv
+    assert int(d.ws[256:256 + 4 * units].sum().item()) == 0
+
+
+def test_bounded_wait_reports_timeout():
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    hhr.hhr_test_wait_timeout(ws, 100_000)
+    assert hhr.hhr_read_status(ws) == hhr.HHR_ERR_TIMEOUT
+    assert hhr.hhr_read_status(ws) == hhr.HHR_OK      # cleared by the read
+    torch.cuda.synchronize()                           # the context is still usable
+
+
+# -------------------------------------------------------------- full sizes
+
+FULL_SAMPLES = {
+    "llama8b_32k": [(0, 0), (0, 5)],
+    "llama8b_128k": [(0, 3), (0, 7)],
+    "batch8_64k_b256": [(0, 0), (5, 2), (7, 7)],
+    "qwen8b_128k_rope": [(1, 4), (3, 0)],
+}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", list(FULL_SAMPLES))
+def test_full_size_sampled_units(name):
+    w = get(name)
+    inp = make_inputs(w)
+    units = FULL_SAMPLES[name]
+    d = Dev(inp)
+    d.encode(0, w.N)
+    codes = np.zeros((w.B, w.Hkv, w.n_cap, w.words), np.uint32)
+    meta = np.zeros((w.B, w.Hkv, w.np_cap, 2, w.d), np.uint16)
+    O.encode_all(inp, 0, w.N, codes=codes, meta=meta, units=units)
+    steps = [0] if not w.appends else list(range(w.appends))
+    for step in steps:
+        if w.appends:
+            d.encode(w.N + step, w.N + step + 1)
+            O.encode_all(inp, w.N + step, w.N + step + 1, codes=codes, meta=meta, units=units)
+        d.decode(step)
+        if step in (0, steps[-1]):
+            ores = O.decode_all(inp, codes, meta, step=step, units=units)
+            rep = compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), units)
+            if rep["page_set_diff"] == 0 and rep["q_ambiguous"] == 0:
+                compare_out(w, ores["out"], _host(d.out), units)
+            print(name, step, rep)
+    assert d.status() == hhr.HHR_OK
+    torch.cuda.synchronize()
+    rep = compare_encode(inp, u32_host(d.codes), bits_host(d.meta), units, inp.n_valid(steps[-1]))
+    print(name, rep)
