@@ -185,6 +185,38 @@ int32_t hhr_decode_step(const hhr_dims* dims, const void* q, const float* R, con
                         int32_t* tok_idx, int32_t* n_sel, float* out, void* workspace,
                         size_t ws_bytes, void* stream);
 
+/* Size of the scratch array hhr_decode_step_noalloc uses (4 MiB). */
+#define HHR_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * hhr_decode_step without a caller workspace.  The paper has no counterpart:
+ * this is a convenience for callers that cannot allocate device memory --
+ * for example code whose device memory is fully managed by another
+ * framework's allocator it cannot reach, or a host program that is not
+ * allowed to allocate after start-up.  The scratch lives in a fixed array of
+ * HHR_NOALLOC_SCRATCH_BYTES inside the library; every device that loads the
+ * library holds that array until the process exits.
+ *   - Arguments and results are those of hhr_decode_step, minus the
+ *     workspace; the caller still passes every input and output buffer.
+ *   - Sizes whose workspace (hhr_workspace_size) exceeds
+ *     HHR_NOALLOC_SCRATCH_BYTES return HHR_ERR_UNSUPPORTED; nothing is
+ *     enqueued.  Other argument errors are reported as hhr_decode_step does.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - The call allocates nothing.  It enqueues a memset of the array's
+ *     status word and counters, then the decode kernel.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents: calls that may overlap on the GPU (different streams without
+ *     ordering) race and give undefined results.  The bounded-wait status of
+ *     this variant cannot be read back; it is cleared by the next call.
+ */
+int32_t hhr_decode_step_noalloc(const hhr_dims* dims, const void* q, const float* R,
+                                const float* W, const uint32_t* codes, const void* meta,
+                                const void* K, const void* V, int32_t n_valid, int32_t P,
+                                int32_t k, float scale, int32_t* page_idx, int32_t* tok_idx,
+                                int32_t* n_sel, float* out, void* stream);
+
 /*
  * Waits for `stream`, returns the workspace status word (HHR_OK or
  * HHR_ERR_TIMEOUT) and clears it.  After HHR_ERR_TIMEOUT the workspace must be

@@ -21,6 +21,7 @@ HHR_ERR_WORKSPACE = 3
 HHR_ERR_CUDA = 4
 HHR_ERR_TIMEOUT = 5
 HHR_MAX_PAGES = 16384
+HHR_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class HhrError(RuntimeError):
@@ -56,6 +57,8 @@ _SIGS = {
                                  C.c_size_t, _P]),
     "hhr_decode_step": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32,
                                C.c_float, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "hhr_decode_step_noalloc": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
+                                       _I32, C.c_float, _P, _P, _P, _P, _P]),
     "hhr_read_status": (_I32, [_P, _P]),
     "hhr_test_wait_timeout": (_I32, [_P, C.c_size_t, C.c_uint64, _P]),
 }
@@ -152,6 +155,15 @@ def hhr_decode_step(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page
                                  _ptr(meta), _ptr(K), _ptr(V), n_valid, P, k, scale,
                                  _ptr(page_idx), _ptr(tok_idx), _ptr(n_sel), _ptr(out),
                                  _ptr(workspace), ws_bytes, _stream(stream)), "hhr_decode_step")
+
+
+def hhr_decode_step_noalloc(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page_idx,
+                            tok_idx, n_sel, out, stream=None) -> None:
+    """hhr_decode_step with the library's built-in scratch (no workspace)."""
+    _check(lib().hhr_decode_step_noalloc(C.byref(dims), _ptr(q), _ptr(R), _ptr(W), _ptr(codes),
+                                         _ptr(meta), _ptr(K), _ptr(V), n_valid, P, k, scale,
+                                         _ptr(page_idx), _ptr(tok_idx), _ptr(n_sel), _ptr(out),
+                                         _stream(stream)), "hhr_decode_step_noalloc")
 
 
 def hhr_read_status(workspace, stream=None) -> int:
