@@ -141,6 +141,7 @@ int32_t finish_launch(cudaError_t e) { return e == cudaSuccess ? HHR_OK : HHR_ER
 
 }  // namespace
 
+
 extern "C" {
 
 int32_t hhr_version(void) { return kVersion; }

@@ -60,13 +60,6 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
   return old;
 }
 
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(d), "l"(gmem_src) : "memory");
@@ -74,6 +67,58 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+
+// 1-D bulk copy global -> shared on the TMA unit; completion is signalled on
+// the mbarrier as transferred bytes.  Both addresses 16-B aligned, size a
+// multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+// Brings the 128-B line holding `p` into L2 (no register result).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+               " selp.u32 %0, 1, 0, p;\n}" : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+  return done != 0;
+}
+
+// Waits for the mbarrier phase with the given parity; gives up (false) after
+// `limit` clock cycles.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long limit) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = clock64();
+  do {
+    if (mbar_try(bar, parity)) return true;
+  } while (static_cast<unsigned long long>(clock64() - t0) <= limit);
+  return false;
+}
+
+// Packed float32 pair multiply-add (one fma.rn.f32x2): d = a * b + c lane-wise.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
 
 // Exclusive prefix sum over the CTA.  Every thread must call it.
 __device__ int block_excl_scan(int v, int* s_warp, int* total) {
@@ -108,6 +153,28 @@ __device__ int block_sum(int v, int* s_warp) {
   int total;
   block_excl_scan(v, s_warp, &total);
   return total;
+}
+
+// For a histogram of kBuckets bins and a count `need` >= 1 not above its
+// total, finds the bin b* holding the need-th largest element (bins ordered
+// by value) and the number of elements in bins above b*.  Thread t owns the
+// four bins [4(NT-1-t), 4(NT-1-t) + 4), so a scan in thread order counts the
+// elements in higher bins.  Every thread must call it; results in out[0..1].
+__device__ void find_boundary(const int* hist, int need, int* s_warp, int* out) {
+  static_assert(kBuckets == 4 * NT, "bin ownership assumes 4 bins per thread");
+  const int base = 4 * (NT - 1 - static_cast<int>(threadIdx.x));
+  const int c4 = hist[base] + hist[base + 1] + hist[base + 2] + hist[base + 3];
+  int tot;
+  int running = block_excl_scan(c4, s_warp, &tot);
+  for (int bin = base + 3; bin >= base; --bin) {
+    const int hcount = hist[bin];
+    if (running < need && running + hcount >= need) {
+      out[0] = bin;
+      out[1] = running;
+    }
+    running += hcount;
+  }
+  __syncthreads();
 }
 
 // Unit barrier: every CTA of the unit adds one to the counter, then waits
@@ -189,61 +256,59 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   const size_t unit_rows = static_cast<size_t>(unit) * a.n_cap;
   const uint16_t* Ku = a.K + unit_rows * kD;
   const uint16_t* Vu = a.V + unit_rows * kD;
-  uint16_t* ring = reinterpret_cast<uint16_t*>(scratch);  // [stages][chunk][2][d]
-  constexpr int STAGE_ELEMS = kAttnChunk * 2 * kD;
 
-  const int n_stages = (cnt + kAttnChunk - 1) / kAttnChunk;
-  auto issue = [&](int s) {
-    if (s < n_stages) {
-      const int tt = tid >> 4, part = tid & 15;  // token in stage, 16-B chunk of its row
-      const int i = s * kAttnChunk + tt;
-      if (i < cnt) {
-        const size_t row = static_cast<size_t>(sel[i]) * kD;
-        uint16_t* dst = ring + (s % kAttnStages) * STAGE_ELEMS + tt * 2 * kD;
-        cp_async16(dst + part * 8, Ku + row + part * 8);
-        cp_async16(dst + kD + part * 8, Vu + row + part * 8);
-      }
+  // Half-warp hw attends tokens sel[hw], sel[hw + 32], ...  Its lane hl only
+  // uses the 16-B slices [8 hl, 8 hl + 8) of each K and V row, so it copies
+  // exactly those into its own slots (kAttnSlots tokens in flight) with
+  // cp.async and waits on its own copies: no barrier is involved.
+  const int hw_id = warp * 2 + hf;
+  uint4* kslot = reinterpret_cast<uint4*>(scratch) + hw_id * kAttnSlots * 16 + hl;
+  uint4* vslot = kslot + 32 * kAttnSlots * 16;
+  const int n_iter = cnt > warp * 2 ? (cnt - warp * 2 + 31) / 32 : 0;  // warp-uniform
+  auto issue_tok = [&](int j) {
+    const int t = hw_id + 32 * j;
+    if (j < n_iter && t < cnt) {
+      const size_t row = static_cast<size_t>(sel[t]) * kD + hl * 8;
+      cp_async16(kslot + (j % kAttnSlots) * 16, Ku + row);
+      cp_async16(vslot + (j % kAttnSlots) * 16, Vu + row);
     }
     cp_async_commit();
   };
 
-  float q[RG][8];
+  float2 q[RG][4];
 #pragma unroll
   for (int h = 0; h < RG; ++h)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) q[h][e] = sq[h * kD + hl * 8 + e];
-  float m[RG], l[RG], o[RG][8];
+    for (int e = 0; e < 4; ++e) q[h][e] = make_float2(sq[h * kD + hl * 8 + 2 * e], sq[h * kD + hl * 8 + 2 * e + 1]);
+  float m[RG], l[RG];
+  float2 o[RG][4];
 #pragma unroll
   for (int h = 0; h < RG; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) o[h][e] = 0.f;
+    for (int e = 0; e < 4; ++e) o[h][e] = make_float2(0.f, 0.f);
   }
 
 #pragma unroll
-  for (int s = 0; s < kAttnStages - 1; ++s) issue(s);
-  for (int s = 0; s < n_stages; ++s) {
-    cp_async_wait<kAttnStages - 2>();
-    __syncthreads();
-    issue(s + kAttnStages - 1);
-    const int ti = warp * 2 + hf;
-    const bool valid = s * kAttnChunk + ti < cnt;   // uniform within a half-warp
-    const uint16_t* rowp = ring + (s % kAttnStages) * STAGE_ELEMS + ti * 2 * kD;
+  for (int j = 0; j < kAttnSlots; ++j) issue_tok(j);
+  for (int j = 0; j < n_iter; ++j) {
+    cp_async_wait<kAttnSlots - 1>();   // this lane's slices of token j have landed
+    const bool valid = hw_id + 32 * j < cnt;   // uniform within a half-warp
     uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
     if (valid) {
-      kv = *reinterpret_cast<const uint4*>(rowp + hl * 8);
-      vv = *reinterpret_cast<const uint4*>(rowp + kD + hl * 8);
+      kv = kslot[(j % kAttnSlots) * 16];
+      vv = vslot[(j % kAttnSlots) * 16];
     }
-    const float kf[8] = {bf_lo(kv.x), bf_hi(kv.x), bf_lo(kv.y), bf_hi(kv.y),
-                         bf_lo(kv.z), bf_hi(kv.z), bf_lo(kv.w), bf_hi(kv.w)};
-    const float vf[8] = {bf_lo(vv.x), bf_hi(vv.x), bf_lo(vv.y), bf_hi(vv.y),
-                         bf_lo(vv.z), bf_hi(vv.z), bf_lo(vv.w), bf_hi(vv.w)};
+    issue_tok(j + kAttnSlots);   // refill the slot just read
+    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+    const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
     for (int h = 0; h < RG; ++h) {
-      float sdot = 0.f;
+      float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sdot = fmaf(q[h][e], kf[e], sdot);
+      for (int e = 0; e < 4; ++e) d2 = ffma2(q[h][e], make_float2(bf_lo(kw[e]), bf_hi(kw[e])), d2);
+      float sdot = d2.x + d2.y;
       // butterfly over the 16 lanes of this half-warp: every lane ends with
       // the same (commutative) sum
       sdot += __shfl_xor_sync(0xFFFFFFFFu, sdot, 8);
@@ -255,13 +320,14 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
           const float alpha = exp2f(m[h] - sdot);
           l[h] *= alpha;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[h][e] *= alpha;
+          for (int e = 0; e < 4; ++e) o[h][e] = make_float2(o[h][e].x * alpha, o[h][e].y * alpha);
           m[h] = sdot;
         }
         const float p = exp2f(sdot - m[h]);
         l[h] += p;
+        const float2 pp = make_float2(p, p);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[h][e] = fmaf(p, vf[e], o[h][e]);
+        for (int e = 0; e < 4; ++e) o[h][e] = ffma2(pp, make_float2(bf_lo(vw[e]), bf_hi(vw[e])), o[h][e]);
       }
     }
   }
@@ -279,9 +345,10 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     const float wb = (M == -INFINITY) ? 0.f : exp2f(mo - M);
     l[h] = l[h] * wa + lo * wb;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float oo = __shfl_xor_sync(0xFFFFFFFFu, o[h][e], 16);
-      o[h][e] = o[h][e] * wa + oo * wb;
+    for (int e = 0; e < 4; ++e) {
+      const float ox = __shfl_xor_sync(0xFFFFFFFFu, o[h][e].x, 16);
+      const float oy = __shfl_xor_sync(0xFFFFFFFFu, o[h][e].y, 16);
+      o[h][e] = make_float2(o[h][e].x * wa + ox * wb, o[h][e].y * wa + oy * wb);
     }
     m[h] = M;
   }
@@ -291,7 +358,10 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     for (int h = 0; h < RG; ++h) {
       float* dst = mer + (warp * RG + h) * (kD + 2);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) dst[hl * 8 + e] = o[h][e];
+      for (int e = 0; e < 4; ++e) {
+        dst[hl * 8 + 2 * e] = o[h][e].x;
+        dst[hl * 8 + 2 * e + 1] = o[h][e].y;
+      }
       if (hl == 0) {
         dst[kD] = m[h];
         dst[kD + 1] = l[h];
@@ -301,7 +371,8 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   __syncthreads();
 
   const int b = unit / a.Hkv, g = unit % a.Hkv;
-  float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * RG * (kD + 2);
+  constexpr int PS = part_stride(RG);
+  float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * PS;
   for (int oi = tid; oi < RG * kD; oi += NT) {
     const int h = oi / kD, j = oi % kD;
     float M = -INFINITY;
@@ -337,18 +408,25 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   if (!s_int[0]) return;
   __threadfence();
   if (a.C > 1) {
-    const float* parts = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit) * RG * (kD + 2);
+    // all C partial states of the unit into shared memory in one pass
+    const float* parts = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit) * PS;
+    float* sp = reinterpret_cast<float*>(scratch);
+    const int n4 = a.C * PS / 4;
+#pragma unroll 4
+    for (int i = tid; i < n4; i += NT)
+      reinterpret_cast<float4*>(sp)[i] = __ldcg(reinterpret_cast<const float4*>(parts) + i);
+    __syncthreads();
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
       float M = -INFINITY;
-      for (int cc = 0; cc < a.C; ++cc) M = fmaxf(M, __ldcg(parts + (cc * RG + h) * (kD + 2) + kD));
+      for (int cc = 0; cc < a.C; ++cc) M = fmaxf(M, sp[cc * PS + h * (kD + 2) + kD]);
       float L = 0.f, O = 0.f;
       if (M != -INFINITY) {
         for (int cc = 0; cc < a.C; ++cc) {
-          const float* src = parts + (cc * RG + h) * (kD + 2);
-          const float wgt = exp2f(__ldcg(src + kD) - M);
-          L = fmaf(__ldcg(src + kD + 1), wgt, L);
-          O = fmaf(__ldcg(src + j), wgt, O);
+          const float* src = sp + cc * PS + h * (kD + 2);
+          const float wgt = exp2f(src[kD] - M);
+          L = fmaf(src[kD + 1], wgt, L);
+          O = fmaf(src[j], wgt, O);
         }
       }
       a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
@@ -378,6 +456,14 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
   S.scratch = smem + lay.scratch;
   int* s_scan = s_int;              // NWARPS + 1 entries
   int* s_misc = s_int + NWARPS + 1; // scalars
+  __shared__ __align__(8) unsigned long long s_rwbar;                       // R / W staging
+  const uint32_t rw_addr = smem_addr(&s_rwbar);
+  uint32_t rw_seq = 0;  // R/W phases used so far
+  if (tid == 0) {
+    mbar_init(rw_addr, 1u);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
 
   for (int unit = blockIdx.x / a.C; unit < a.units; unit += a.grid_units) {
     const int b = unit / a.Hkv, g = unit % a.Hkv;
@@ -393,6 +479,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       const int s0 = static_cast<int>(static_cast<long long>(c) * n / a.C);
       const int s1 = static_cast<int>(static_cast<long long>(c + 1) * n / a.C);
       const int32_t* src = a.tok_in + static_cast<size_t>(unit) * a.k;
+#pragma unroll 8
       for (int i = s0 + tid; i < s1; i += NT) S.sel[i - s0] = src[i];
       for (int i = tid; i < RG * kD; i += NT) S.qf[i] *= a.scale_log2;
       __syncthreads();
@@ -402,68 +489,163 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       continue;
     } else {
       // ---------------------------------------------------------- phase 0
+      // R (and later W) reach shared memory by one bulk copy on their own
+      // mbarrier, requested before any metadata so that q~ = q R is ready
+      // first.  Each warp then streams its own slice of pages.
+      const long long pb = static_cast<long long>(c) * a.NP / a.C;
+      const long long pe = static_cast<long long>(c + 1) * a.NP / a.C;
+      const int my_pages = static_cast<int>(pe - pb);
+      float* sRW = reinterpret_cast<float*>(S.scratch + NWARPS * kLaneSlots * 512);
       const float* Rg = a.R + static_cast<size_t>(g) * kD * kD;
+      const float* Wg = a.W + static_cast<size_t>(g) * kD * BITS;
+      auto issue_w = [&](int half_w) {  // thread 0 only: 128 columns of W
+        mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
+        if constexpr (BITS == kD) {
+          bulk_g2s(smem_addr(sRW), Wg, kD * kD * sizeof(float), rw_addr);
+        } else {
+          for (int i = 0; i < kD; ++i)
+            bulk_g2s(smem_addr(sRW + i * kD), Wg + static_cast<size_t>(i) * BITS + half_w * kD,
+                     kD * sizeof(float), rw_addr);
+        }
+      };
+      // thread 0 waits for the next R/W phase; false (all threads) on timeout
+      auto wait_rw = [&]() {
+        const bool ok = (tid == 0) ? mbar_wait(rw_addr, rw_seq & 1u, a.spin_limit) : true;
+        ++rw_seq;
+        return !__syncthreads_or(!ok);
+      };
+
+      // This warp's pages [wpb, wpe).  Lane l only ever reads bytes
+      // [16 l, 16 l + 16) of a page, so it copies exactly those bytes into its
+      // own shared-memory slots with cp.async and waits on its own copies: no
+      // barrier is involved.  kLaneSlots pages are in flight per warp.
+      const long long wpb = pb + static_cast<long long>(my_pages) * warp / NWARPS;
+      const long long wpe = pb + static_cast<long long>(my_pages) * (warp + 1) / NWARPS;
+      const int w_pages = static_cast<int>(wpe - wpb);
+      const int n_grp = (w_pages + kPagesPerGroup - 1) / kPagesPerGroup;
+      const uint16_t* meta_u = a.meta + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
+      const uint4* wsrc = reinterpret_cast<const uint4*>(meta_u + wpb * 2 * kD) + lane;  // 32 x 16 B per page
+      uint4* lslots = reinterpret_cast<uint4*>(S.scratch) + warp * kLaneSlots * 32 + lane;
+      auto issue_group = [&](int gi) {  // every lane: its 16 B of four pages, one commit group
+        if (gi < n_grp) {
+#pragma unroll
+          for (int pp = 0; pp < kPagesPerGroup; ++pp) {
+            const int pg = gi * kPagesPerGroup + pp;
+            if (pg < w_pages) cp_async16(lslots + (pg % kLaneSlots) * 32, wsrc + static_cast<size_t>(pg) * 32);
+          }
+        }
+        cp_async_commit();
+      };
+
+      if (tid == 0) {
+        mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
+        bulk_g2s(smem_addr(sRW), Rg, kD * kD * sizeof(float), rw_addr);
+      }
+#pragma unroll
+      for (int gi = 0; gi < kLaneSlots / kPagesPerGroup; ++gi) issue_group(gi);
+      if (!wait_rw()) {
+        cp_async_wait<0>();
+        if (tid == 0) {
+          atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+          mbar_wait(rw_addr, (rw_seq - 1) & 1u, a.spin_limit);
+        }
+        __syncthreads();
+        return;
+      }
       for (int oi = tid; oi < RG * kD; oi += NT) {
         const int h = oi / kD, j = oi % kD;
-        float acc = 0.f;
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll 8
-        for (int i = 0; i < kD; ++i) acc = fmaf(S.qf[h * kD + i], __ldg(Rg + i * kD + j), acc);
-        S.qt[oi] = acc;
+        for (int i = 0; i < kD; i += 2)
+          acc = ffma2(make_float2(S.qf[h * kD + i], S.qf[h * kD + i + 1]),
+                      make_float2(sRW[i * kD + j], sRW[(i + 1) * kD + j]), acc);
+        S.qt[oi] = acc.x + acc.y;
       }
       __syncthreads();
+      // the first 128 columns of W stream in while the page bounds run
+      if (tid == 0) issue_w(0);
 
       // ---------------------------------------------------------- phase 1
-      constexpr int PPI = (RG == 1) ? 8 : 16 / RG;  // pages per warp iteration
-      constexpr int NV = PPI * RG;
+      // Warp-per-page scoring.  A 512-B page is one 16-B load per lane: lanes
+      // 0-15 read lower bounds and hold min(q~, 0), lanes 16-31 read upper
+      // bounds and hold max(q~, 0), so Eq. 3 is one multiply-add per stored
+      // bound.  A stage's four pages x r heads partial sums are folded with a
+      // butterfly reduce-scatter, then the max over the heads is taken.
+      constexpr int NV = kPagesPerGroup * RG;
       constexpr int LNV = Log2<NV>::value;
       constexpr int SH = 5 - LNV;                   // lanes sharing one value index
+      static_assert(NV <= 32, "at most 32 partial sums per lane");
       const int half = lane >> 4, dl = (lane & 15) * 8;
-      float qs[RG][8];
+      float2 qs[RG][4];
 #pragma unroll
       for (int h = 0; h < RG; ++h)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float v = S.qt[h * kD + dl + e];
-          qs[h][e] = half ? fmaxf(v, 0.f) : fminf(v, 0.f);
+        for (int e = 0; e < 4; ++e) {
+          const float v0 = S.qt[h * kD + dl + 2 * e], v1 = S.qt[h * kD + dl + 2 * e + 1];
+          qs[h][e] = half ? make_float2(fmaxf(v0, 0.f), fmaxf(v1, 0.f))
+                          : make_float2(fminf(v0, 0.f), fminf(v1, 0.f));
         }
-      const long long pb = static_cast<long long>(c) * a.NP / a.C;
-      const long long pe = static_cast<long long>(c + 1) * a.NP / a.C;
-      const uint16_t* meta_u = a.meta + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
       float* wsU_u = a.wsU + static_cast<size_t>(unit) * a.np_stride;
       float lmin = INFINITY, lmax = -INFINITY;
-      for (long long p0 = pb + static_cast<long long>(warp) * PPI; p0 < pe;
-           p0 += static_cast<long long>(NWARPS) * PPI) {
-        uint4 x[PPI];
-#pragma unroll
-        for (int i = 0; i < PPI; ++i) {
-          if (p0 + i < pe) x[i] = ld_stream16(meta_u + (p0 + i) * 2 * kD + lane * 8);
-          else x[i] = make_uint4(0u, 0u, 0u, 0u);
-        }
+      for (int gi = 0; gi < n_grp; ++gi) {
+        cp_async_wait<kLaneSlots / kPagesPerGroup - 1>();   // this lane's group gi has landed
+        const int spages = min(kPagesPerGroup, w_pages - gi * kPagesPerGroup);
         float v[NV];
 #pragma unroll
-        for (int i = 0; i < PPI; ++i) {
-          const float xf[8] = {bf_lo(x[i].x), bf_hi(x[i].x), bf_lo(x[i].y), bf_hi(x[i].y),
-                               bf_lo(x[i].z), bf_hi(x[i].z), bf_lo(x[i].w), bf_hi(x[i].w)};
+        for (int pp = 0; pp < kPagesPerGroup; ++pp) {
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (pp < spages) x = lslots[((gi * kPagesPerGroup + pp) % kLaneSlots) * 32];
+          const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
           for (int h = 0; h < RG; ++h) {
-            float acc = 0.f;
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc = fmaf(qs[h][e], xf[e], acc);
-            v[i * RG + h] = acc;
+            for (int e = 0; e < 4; ++e) acc = ffma2(qs[h][e], make_float2(bf_lo(xw[e]), bf_hi(xw[e])), acc);
+            v[pp * RG + h] = acc.x + acc.y;
           }
         }
+        issue_group(gi + kLaneSlots / kPagesPerGroup);  // refill the slots just read
         reduce_scatter<NV>(v, lane);
         const int idx = lane >> SH;
         float u = v[0];
 #pragma unroll
         for (int mm = 1; mm < RG; mm <<= 1) u = fmaxf(u, __shfl_xor_sync(0xFFFFFFFFu, u, mm << SH));
-        const long long p = p0 + idx / RG;
-        if ((idx % RG) == 0 && (lane & ((1 << SH) - 1)) == 0 && p < pe) {
-          wsU_u[p] = u;
-          if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + p] = u;
+        const int pl = idx / RG;
+        if ((idx % RG) == 0 && (lane & ((1 << SH) - 1)) == 0 && pl < spages) {
+          const long long pg = wpb + static_cast<long long>(gi) * kPagesPerGroup + pl;
+          wsU_u[pg] = u;
+          if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
           lmin = fminf(lmin, u);
           lmax = fmaxf(lmax, u);
         }
+      }
+      cp_async_wait<0>();
+      // query codes (Eq. 10 + sign) from W in shared memory, 128 columns at
+      // a time
+      int w_done = 0;
+      bool q_ok = true;
+      while (q_ok && w_done < BITS / kD) {
+        q_ok = wait_rw();
+        if (!q_ok) break;
+        for (int oi = tid; oi < RG * kD; oi += NT) {  // warp-uniform trip count
+          const int h = oi / kD, t = oi % kD;
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 8
+          for (int i = 0; i < kD; i += 2)
+            acc = ffma2(make_float2(S.qf[h * kD + i], S.qf[h * kD + i + 1]),
+                        make_float2(sRW[i * kD + t], sRW[(i + 1) * kD + t]), acc);
+          const uint32_t word = __ballot_sync(0xFFFFFFFFu, acc.x + acc.y > 0.f);
+          if (lane == 0) S.qc[h * WORDS + w_done * (kD / 32) + t / 32] = word;
+        }
+        ++w_done;
+        if (w_done < BITS / kD) {
+          __syncthreads();
+          if (tid == 0) issue_w(w_done);
+        }
+      }
+      if (__syncthreads_or(!q_ok)) {
+        if (tid == 0) atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+        return;
       }
       // CTA min / max of its bounds
 #pragma unroll
@@ -494,17 +676,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         __threadfence();
         atom_add_acq_rel(ctr, 1u);
       }
-      {
-        const float* Wg = a.W + static_cast<size_t>(g) * kD * BITS;
-        for (int oi = tid; oi < RG * BITS; oi += NT) {  // warp-uniform trip count
-          const int h = oi / BITS, t = oi % BITS;
-          float acc = 0.f;
-#pragma unroll 8
-          for (int i = 0; i < kD; ++i) acc = fmaf(S.qf[h * kD + i], __ldg(Wg + i * BITS + t), acc);
-          const uint32_t word = __ballot_sync(0xFFFFFFFFu, acc > 0.f);
-          if (lane == 0) S.qc[h * WORDS + t / 32] = word;
-        }
-      }
       if (tid == 0) {
         int ok = 1;
         const long long t0 = clock64();
@@ -530,7 +701,15 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       const int nwords = (NP + 31) / 32;
       float* sCU = reinterpret_cast<float*>(sBits + align_up(nwords, 4));
       int* sCP = reinterpret_cast<int*>(sCU + kCandMax);
-      for (int p = tid; p < NP; p += NT) sU[p] = __ldcg(wsU_u + p);
+      float* sC2U = reinterpret_cast<float*>(sCP + kCandMax);
+      int* sC2P = reinterpret_cast<int*>(sC2U + kCandMax);
+      {
+        const int n4 = NP / 4;
+        const float4* src4 = reinterpret_cast<const float4*>(wsU_u);
+#pragma unroll 4
+        for (int i = tid; i < n4; i += NT) reinterpret_cast<float4*>(sU)[i] = __ldcg(src4 + i);
+        for (int p = n4 * 4 + tid; p < NP; p += NT) sU[p] = __ldcg(wsU_u + p);
+      }
       for (int i = tid; i < kBuckets; i += NT) sHist[i] = 0;
       for (int i = tid; i < nwords; i += NT) sBits[i] = 0u;
       if (warp == 0) {
@@ -568,22 +747,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         };
         for (int p = tid; p < NP; p += NT) atomicAdd(&sHist[bucket(sU[p])], 1);
         __syncthreads();
-        // thread t owns the four bins [4(NT-1-t), 4(NT-1-t)+4): a scan in
-        // thread order counts the pages in higher bins
-        static_assert(kBuckets == 4 * NT, "bin ownership assumes 4 bins per thread");
-        const int base = 4 * (NT - 1 - tid);
-        const int c4 = sHist[base] + sHist[base + 1] + sHist[base + 2] + sHist[base + 3];
-        int tot;
-        int running = block_excl_scan(c4, s_scan, &tot);
-        for (int bin = base + 3; bin >= base; --bin) {
-          const int hcount = sHist[bin];
-          if (running < Pk && running + hcount >= Pk) {
-            s_misc[3] = bin;
-            s_misc[4] = running;
-          }
-          running += hcount;
-        }
-        __syncthreads();
+        find_boundary(sHist, Pk, s_scan, &s_misc[3]);
         const int bstar = s_misc[3];
         const int need = Pk - s_misc[4];
         const int cntB = sHist[bstar];
@@ -606,16 +770,72 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
             }
           }
           __syncthreads();
-          const int nc = s_misc[2];
+          int nc = s_misc[2];
+          int need2 = need;
+          const float* fu = sCU;
+          const int* fp = sCP;
+          if (nc > kRankDirect) {
+            // second level: linear bins over the boundary bin's own range
+            float mn = INFINITY, mx = -INFINITY;
+            for (int i = tid; i < nc; i += NT) {
+              mn = fminf(mn, sCU[i]);
+              mx = fmaxf(mx, sCU[i]);
+            }
+#pragma unroll
+            for (int o2 = 16; o2 >= 1; o2 >>= 1) {
+              mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o2));
+              mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o2));
+            }
+            float* red2 = reinterpret_cast<float*>(sC2P + kCandMax);
+            if (lane == 0) {
+              red2[warp] = mn;
+              red2[NWARPS + warp] = mx;
+            }
+            for (int i = tid; i < kBuckets; i += NT) sHist[i] = 0;
+            if (tid == 0) s_misc[2] = 0;
+            __syncthreads();
+            float cmin = INFINITY, cmax = -INFINITY;
+            for (int w2 = 0; w2 < NWARPS; ++w2) {
+              cmin = fminf(cmin, red2[w2]);
+              cmax = fmaxf(cmax, red2[NWARPS + w2]);
+            }
+            const float r2 = cmax - cmin;
+            const float inv2 = (r2 > 0.f && r2 <= FLT_MAX) ? static_cast<float>(kBuckets) / r2 : 0.f;
+            auto bucket2 = [&](float u) {
+              const int bk = static_cast<int>((u - cmin) * inv2);
+              return bk < kBuckets - 1 ? bk : kBuckets - 1;
+            };
+            for (int i = tid; i < nc; i += NT) atomicAdd(&sHist[bucket2(sCU[i])], 1);
+            __syncthreads();
+            find_boundary(sHist, need, s_scan, &s_misc[5]);
+            const int b2 = s_misc[5];
+            need2 = need - s_misc[6];
+            for (int i = tid; i < nc; i += NT) {
+              const int bk = bucket2(sCU[i]);
+              if (bk > b2) {
+                atomicOr(&sBits[sCP[i] >> 5], 1u << (sCP[i] & 31));
+              } else if (bk == b2) {
+                const int slot = atomicAdd(&s_misc[2], 1);
+                sC2U[slot] = sCU[i];
+                sC2P[slot] = sCP[i];
+              }
+            }
+            __syncthreads();
+            nc = s_misc[2];
+            fu = sC2U;
+            fp = sC2P;
+          }
+          // exact ranking of the remaining boundary pages: larger bound first,
+          // then lower page index
           for (int i = tid; i < nc; i += NT) {
-            const float u = sCU[i];
-            const int pi = sCP[i];
+            const float u = fu[i];
+            const int pi = fp[i];
             int rank = 0;
             for (int j = 0; j < nc; ++j) {
-              const float uj = sCU[j];
-              rank += (uj > u) || (uj == u && sCP[j] < pi);
+              const float uj = fu[j];
+              rank += (uj > u) || (uj == u && fp[j] < pi);
             }
-            if (rank < need) atomicOr(&sBits[pi >> 5], 1u << (pi & 31));
+            if (rank < need2) atomicOr(&sBits[pi >> 5], 1u << (pi & 31));
           }
         } else {
           // many equal-looking bounds: exact search for the Pk-th largest key
@@ -649,15 +869,19 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       const int ks = static_cast<int>(static_cast<long long>(c) * Pk / a.C);
       const int ke = static_cast<int>(static_cast<long long>(c + 1) * Pk / a.C);
       {
-        const int span = (NP + NT - 1) / NT;
-        const int lo = tid * span, hi = min(NP, lo + span);
+        // thread t owns bitmap words [t*wpt, (t+1)*wpt)
+        const int wpt = (nwords + NT - 1) / NT;
+        const int w0 = tid * wpt, w1 = min(nwords, w0 + wpt);
         int cnt = 0;
-        for (int p = lo; p < hi; ++p) cnt += (sBits[p >> 5] >> (p & 31)) & 1u;
+        for (int wi = w0; wi < w1; ++wi) cnt += __popc(sBits[wi]);
         int tot;
         int pos = block_excl_scan(cnt, s_scan, &tot);
         int32_t* pidx = a.page_idx + static_cast<size_t>(unit) * a.P;
-        for (int p = lo; p < hi; ++p) {
-          if ((sBits[p >> 5] >> (p & 31)) & 1u) {
+        for (int wi = w0; wi < w1; ++wi) {
+          uint32_t bits = sBits[wi];
+          while (bits) {
+            const int p = wi * 32 + __ffs(bits) - 1;
+            bits &= bits - 1u;
             if (pos >= ks && pos < ke) S.my_pages[pos - ks] = p;
             if (c == 0) pidx[pos] = p;
             ++pos;
@@ -723,12 +947,73 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         int32_t* hrow = a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * (BITS + 1);
         for (int i = tid; i <= BITS; i += NT) hrow[i] = sHD[i];
       }
-      if (!unit_arrive_wait(ctr, 2u * a.C, a, &s_misc[0])) return;
+      // unit barrier 2.  While waiting, a fused step prefetches into L2 the
+      // K/V rows of the tokens it most likely keeps: those at or below the
+      // local distance quantile k / (kept tokens), the fraction the global
+      // threshold keeps.  Prefetching changes no result.
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        atom_add_acq_rel(ctr, 1u);
+      }
+      if constexpr (MODE == kModeFused) {
+        if (warp == 0) {
+          int local = 0;
+          for (int v = lane; v <= BITS; v += 32) local += sHD[v];
+#pragma unroll
+          for (int o2 = 16; o2 >= 1; o2 >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, o2);
+          const long long cand = static_cast<long long>(Pk) * S_;
+          const long long target = cand > 0 ? (static_cast<long long>(local) * a.k + cand - 1) / cand : 0;
+          int t_loc = -1, run = 0;
+          for (int v0 = 0; v0 <= BITS && t_loc < 0; v0 += 32) {
+            int x = (v0 + lane <= BITS) ? sHD[v0 + lane] : 0;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+              const int y = __shfl_up_sync(0xFFFFFFFFu, x, o2);
+              if (lane >= o2) x += y;
+            }
+            const unsigned hit = __ballot_sync(0xFFFFFFFFu, run + x >= target && target > 0);
+            if (hit) t_loc = v0 + __ffs(hit) - 1;
+            run += __shfl_sync(0xFFFFFFFFu, x, 31);
+          }
+          if (lane == 0) s_misc[10] = (target >= local) ? BITS : t_loc;
+        }
+        __syncthreads();
+        const int t_loc = s_misc[10];
+        const size_t unit_rows = static_cast<size_t>(unit) * a.n_cap;
+        for (int i = tid; i < ntok; i += NT) {
+          if (static_cast<int>(S.tokD[i]) <= t_loc) {
+            const int slot = i / S_;
+            const size_t n = static_cast<size_t>(S.my_pages[slot]) * S_ + (i - slot * S_);
+            prefetch_l2(a.K + (unit_rows + n) * kD);
+            prefetch_l2(a.K + (unit_rows + n) * kD + 64);
+            prefetch_l2(a.V + (unit_rows + n) * kD);
+            prefetch_l2(a.V + (unit_rows + n) * kD + 64);
+          }
+        }
+      }
+      if (tid == 0) {
+        int ok = 1;
+        const long long t0 = clock64();
+        while (ld_acquire(ctr) < 2u * static_cast<uint32_t>(a.C)) {
+          if (static_cast<unsigned long long>(clock64() - t0) > a.spin_limit) {
+            atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+            ok = 0;
+            break;
+          }
+          __nanosleep(32);
+        }
+        __threadfence();
+        s_misc[0] = ok;
+      }
+      __syncthreads();
+      if (!s_misc[0]) return;
 
       // ---------------------------------------------------------- phase 5
       int* sHA = reinterpret_cast<int*>(S.scratch);  // [C][BITS + 1]
       {
         const int32_t* hall = a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit) * (BITS + 1);
+#pragma unroll 8
         for (int i = tid; i < a.C * (BITS + 1); i += NT) sHA[i] = __ldcg(hall + i);
       }
       __syncthreads();
@@ -752,11 +1037,15 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       const int needT = s_misc[6];
       int* sBelow = s_aux;
       int* sEq = s_aux + kMaxCtasPerUnit;
-      if (tid < a.C) {
+      for (int cc = warp; cc < a.C; cc += NWARPS) {  // one warp per CTA row
         int below = 0;
-        for (int v = 0; v < T; ++v) below += sHA[tid * (BITS + 1) + v];
-        sBelow[tid] = below;
-        sEq[tid] = T >= 0 ? sHA[tid * (BITS + 1) + T] : 0;
+        for (int v = lane; v < T; v += 32) below += sHA[cc * (BITS + 1) + v];
+#pragma unroll
+        for (int o2 = 16; o2 >= 1; o2 >>= 1) below += __shfl_xor_sync(0xFFFFFFFFu, below, o2);
+        if (lane == 0) {
+          sBelow[cc] = below;
+          sEq[cc] = T >= 0 ? sHA[cc * (BITS + 1) + T] : 0;
+        }
       }
       __syncthreads();
       if (tid == 0) {

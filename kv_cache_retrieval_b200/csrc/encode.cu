@@ -31,6 +31,7 @@ struct EncSmem {
 
 __device__ __forceinline__ void load_operand(float (*bm)[kPadB], const float* src, int ld) {
   // 128 x 128 floats, row stride `ld` floats in global memory
+#pragma unroll 16
   for (int idx = threadIdx.x; idx < kD * kD / 4; idx += kEncThreads) {
     const int i = idx / (kD / 4), j4 = idx % (kD / 4);
     const float4 v = __ldg(reinterpret_cast<const float4*>(src + static_cast<size_t>(i) * ld) + j4);
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const EncodeArgs
   const uint16_t* Ku = a.K + unit_rows * kD;
 
   // key tile, transposed to [dim][row]; rows outside [n_begin, n_end) are 0
+#pragma unroll 4
   for (int idx = threadIdx.x; idx < kTile * (kD / 8); idx += kEncThreads) {
     const int row = idx / (kD / 8), c8 = idx % (kD / 8);
     const int n = t0 + row;

@@ -15,13 +15,19 @@ constexpr int kDecodeThreads = 512;     // one decode CTA per SM, 16 warps
 constexpr int kMaxCtasPerUnit = 64;     // CTAs that may share one (sequence, KV head)
 constexpr int kMinPagesPerCta = 32;     // below this a unit uses fewer CTAs
 constexpr int kBuckets = 2048;          // page top-P histogram bins
-constexpr int kCandMax = 1024;          // boundary-bucket candidates ranked exactly
+constexpr int kCandMax = 1024;          // boundary-bucket candidates held in shared memory
+constexpr int kRankDirect = 48;         // at most this many are ranked without a second level
 constexpr int kMaxTokensPerCta = 16384; // candidate tokens one CTA scores
-constexpr int kAttnChunk = 32;          // tokens per K/V staging stage
-constexpr int kAttnStages = 4;          // depth of the K/V staging ring
+constexpr int kAttnSlots = 8;           // K/V tokens in flight per half-warp
+constexpr int kPagesPerGroup = 4;      // pages a warp scores per step (one copy group)
+constexpr int kLaneSlots = 16;         // pages in flight per warp (8 KiB)
 constexpr unsigned long long kSpinLimit = 1ull << 31;  // ~1 s at 2 GHz
 
 inline __host__ __device__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Floats of one CTA's partial softmax state (r heads x (d outputs, max, sum)),
+// padded to a multiple of four so it can be moved with 16-B accesses.
+inline __host__ __device__ constexpr int part_stride(int r) { return (r * (kD + 2) + 3) / 4 * 4; }
 
 // Workspace layout (bytes).  The status word sits at offset 0.
 struct WsLayout {
@@ -38,7 +44,7 @@ inline __host__ __device__ WsLayout ws_layout(int units, int np_cap, int r, int 
   L.U = off;        off += align_up(sizeof(float) * (size_t)units * L.np_stride, 256);
   L.minmax = off;   off += align_up(sizeof(float) * 2 * (size_t)units * kMaxCtasPerUnit, 256);
   L.hist = off;     off += align_up(sizeof(int32_t) * (size_t)units * kMaxCtasPerUnit * (bits + 1), 256);
-  L.part = off;     off += align_up(sizeof(float) * (size_t)units * kMaxCtasPerUnit * r * (kD + 2), 256);
+  L.part = off;     off += align_up(sizeof(float) * (size_t)units * kMaxCtasPerUnit * part_stride(r), 256);
   L.total = off;
   return L;
 }
@@ -94,20 +100,26 @@ struct DecodeSmem {
 };
 
 inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, int r, int mode) {
-  size_t sel = 0, hist = 0, attn = 0;
+  size_t sel = 0, hist = 0, attn = 0, stream = 0;
   if (mode != kModeAttend) {
+    // per-warp metadata rings + R / W staging (phases 0-1)
+    stream = (size_t)(kDecodeThreads / 32) * kLaneSlots * 512 + sizeof(float) * kD * kD;
     sel = sizeof(float) * align_up((size_t)NP, 4)          // U of every page
         + sizeof(int) * kBuckets                             // histogram
         + sizeof(uint32_t) * align_up(((size_t)NP + 31) / 32, 4)  // kept bitmap
-        + (sizeof(float) + sizeof(int)) * kCandMax;          // boundary candidates
+        + 2 * (sizeof(float) + sizeof(int)) * kCandMax       // boundary candidates, 2 levels
+        + sizeof(float) * 2 * (kDecodeThreads / 32);          // level-2 min / max
     hist = sizeof(int) * (size_t)C * (bits + 1) + 16;
   }
   if (mode != kModeSelect) {
-    const size_t ring = (size_t)kAttnStages * kAttnChunk * 2 * kD * sizeof(uint16_t);
-    const size_t merge = sizeof(float) * (kDecodeThreads / 32) * (size_t)r * (kD + 2);
+    const size_t ring = (size_t)32 * kAttnSlots * 16 * 2 * 16;  // half-warps x slots x lanes x (K, V) x 16 B
+    size_t merge = sizeof(float) * (kDecodeThreads / 32) * (size_t)r * (kD + 2);
+    const size_t parts = sizeof(float) * (size_t)C * part_stride(r);  // final merge
+    merge = merge > parts ? merge : parts;
     attn = ring > merge ? ring : merge;
   }
   size_t m = sel > hist ? sel : hist;
+  m = m > stream ? m : stream;
   return m > attn ? m : attn;
 }
 
