@@ -155,6 +155,42 @@ __device__ int block_sum(int v, int* s_warp) {
   return total;
 }
 
+__device__ __forceinline__ uint32_t order_key(float u) {
+  const uint32_t x = __float_as_uint(u + 0.0f);  // -0 -> +0
+  return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
+}
+
+// Exact top-`Pk` of the NP bounds in sU, ties to the lower page index, as a
+// bitmap: a 32-step bitwise search for the Pk-th largest order key, then a
+// page-order scan for the ties.  Used only when very many bounds fall into
+// one histogram bin (degenerate inputs), so it is kept out of line.
+__device__ __noinline__ void exact_top_pages(const float* sU, int NP, int Pk, int* s_scan,
+                                             uint32_t* sBits) {
+  const int tid = threadIdx.x;
+  uint32_t T = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int cnt = 0;
+    for (int p = tid; p < NP; p += NT) cnt += order_key(sU[p]) >= cand;
+    if (block_sum(cnt, s_scan) >= Pk) T = cand;
+  }
+  int gt = 0;
+  for (int p = tid; p < NP; p += NT) gt += order_key(sU[p]) > T;
+  const int need_eq = Pk - block_sum(gt, s_scan);
+  const int span = (NP + NT - 1) / NT;
+  const int lo = tid * span, hi = min(NP, lo + span);
+  int eq = 0;
+  for (int p = lo; p < hi; ++p) eq += order_key(sU[p]) == T;
+  int eqtot;
+  int er = block_excl_scan(eq, s_scan, &eqtot);
+  for (int p = lo; p < hi; ++p) {
+    const uint32_t kk = order_key(sU[p]);
+    bool keep = kk > T;
+    if (kk == T) keep = (er++ < need_eq);
+    if (keep) atomicOr(&sBits[p >> 5], 1u << (p & 31));
+  }
+}
+
 // For a histogram of kBuckets bins and a count `need` >= 1 not above its
 // total, finds the bin b* holding the need-th largest element (bins ordered
 // by value) and the number of elements in bins above b*.  Thread t owns the
@@ -229,10 +265,6 @@ struct Log2 {
   static constexpr int value = (NV >= 32) ? 5 : (NV >= 16) ? 4 : (NV >= 8) ? 3 : (NV >= 4) ? 2 : (NV >= 2) ? 1 : 0;
 };
 
-__device__ __forceinline__ uint32_t order_key(float u) {
-  const uint32_t x = __float_as_uint(u + 0.0f);  // -0 -> +0
-  return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
-}
 
 struct Smem {
   float* qt;       // [r][d] rotated queries
@@ -265,12 +297,17 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   uint4* kslot = reinterpret_cast<uint4*>(scratch) + hw_id * kAttnSlots * 16 + hl;
   uint4* vslot = kslot + 32 * kAttnSlots * 16;
   const int n_iter = cnt > warp * 2 ? (cnt - warp * 2 + 31) / 32 : 0;  // warp-uniform
-  auto issue_tok = [&](int j) {
-    const int t = hw_id + 32 * j;
-    if (j < n_iter && t < cnt) {
-      const size_t row = static_cast<size_t>(sel[t]) * kD + hl * 8;
-      cp_async16(kslot + (j % kAttnSlots) * 16, Ku + row);
-      cp_async16(vslot + (j % kAttnSlots) * 16, Vu + row);
+  const int n_pair = (n_iter + 1) / 2;
+  auto issue_pair = [&](int jp) {  // tokens 2 jp and 2 jp + 1 of this half-warp: one group
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = 2 * jp + u;
+      const int t = hw_id + 32 * j;
+      if (j < n_iter && t < cnt) {
+        const size_t row = static_cast<size_t>(sel[t]) * kD + hl * 8;
+        cp_async16(kslot + (j % kAttnSlots) * 16, Ku + row);
+        cp_async16(vslot + (j % kAttnSlots) * 16, Vu + row);
+      }
     }
     cp_async_commit();
   };
@@ -291,43 +328,54 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   }
 
 #pragma unroll
-  for (int j = 0; j < kAttnSlots; ++j) issue_tok(j);
-  for (int j = 0; j < n_iter; ++j) {
-    cp_async_wait<kAttnSlots - 1>();   // this lane's slices of token j have landed
-    const bool valid = hw_id + 32 * j < cnt;   // uniform within a half-warp
-    uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
-    if (valid) {
-      kv = kslot[(j % kAttnSlots) * 16];
-      vv = vslot[(j % kAttnSlots) * 16];
+  for (int jp = 0; jp < kAttnSlots / 2; ++jp) issue_pair(jp);
+  for (int jp = 0; jp < n_pair; ++jp) {
+    cp_async_wait<kAttnSlots / 2 - 1>();   // this lane's slices of the pair have landed
+    const int j0 = 2 * jp;
+    const bool va = hw_id + 32 * j0 < cnt;          // uniform within a half-warp
+    const bool vb = hw_id + 32 * (j0 + 1) < cnt;
+    uint4 ka = make_uint4(0u, 0u, 0u, 0u), kb = ka, xa = ka, xb = ka;
+    if (va) {
+      ka = kslot[(j0 % kAttnSlots) * 16];
+      xa = vslot[(j0 % kAttnSlots) * 16];
     }
-    issue_tok(j + kAttnSlots);   // refill the slot just read
-    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-    const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+    if (vb) {
+      kb = kslot[((j0 + 1) % kAttnSlots) * 16];
+      xb = vslot[((j0 + 1) % kAttnSlots) * 16];
+    }
+    issue_pair(jp + kAttnSlots / 2);   // refill the slots just read
+    const uint32_t kwa[4] = {ka.x, ka.y, ka.z, ka.w}, kwb[4] = {kb.x, kb.y, kb.z, kb.w};
+    const uint32_t vwa[4] = {xa.x, xa.y, xa.z, xa.w}, vwb[4] = {xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
     for (int h = 0; h < RG; ++h) {
-      float2 d2 = make_float2(0.f, 0.f);
+      float2 da = make_float2(0.f, 0.f), db = da;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) d2 = ffma2(q[h][e], make_float2(bf_lo(kw[e]), bf_hi(kw[e])), d2);
-      float sdot = d2.x + d2.y;
-      // butterfly over the 16 lanes of this half-warp: every lane ends with
-      // the same (commutative) sum
-      sdot += __shfl_xor_sync(0xFFFFFFFFu, sdot, 8);
-      sdot += __shfl_xor_sync(0xFFFFFFFFu, sdot, 4);
-      sdot += __shfl_xor_sync(0xFFFFFFFFu, sdot, 2);
-      sdot += __shfl_xor_sync(0xFFFFFFFFu, sdot, 1);
-      if (valid) {
-        if (sdot > m[h]) {
-          const float alpha = exp2f(m[h] - sdot);
-          l[h] *= alpha;
+      for (int e = 0; e < 4; ++e) {
+        da = ffma2(q[h][e], make_float2(bf_lo(kwa[e]), bf_hi(kwa[e])), da);
+        db = ffma2(q[h][e], make_float2(bf_lo(kwb[e]), bf_hi(kwb[e])), db);
+      }
+      float sa = da.x + da.y, sb = db.x + db.y;
+      // butterflies over the 16 lanes of this half-warp: every lane ends
+      // with the same (commutative) sums
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[h][e] = make_float2(o[h][e].x * alpha, o[h][e].y * alpha);
-          m[h] = sdot;
+      for (int o2 = 8; o2 >= 1; o2 >>= 1) {
+        sa += __shfl_xor_sync(0xFFFFFFFFu, sa, o2);
+        sb += __shfl_xor_sync(0xFFFFFFFFu, sb, o2);
+      }
+      const float mn = fmaxf(m[h], fmaxf(va ? sa : -INFINITY, vb ? sb : -INFINITY));
+      if (mn != -INFINITY) {
+        const float alpha = exp2f(m[h] - mn);      // 0 when m was -inf
+        const float pa = va ? exp2f(sa - mn) : 0.f;
+        const float pb = vb ? exp2f(sb - mn) : 0.f;
+        l[h] = fmaf(l[h], alpha, pa + pb);
+        const float2 al = make_float2(alpha, alpha), p2a = make_float2(pa, pa), p2b = make_float2(pb, pb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 t2 = make_float2(o[h][e].x * al.x, o[h][e].y * al.y);
+          t2 = ffma2(p2a, make_float2(bf_lo(vwa[e]), bf_hi(vwa[e])), t2);
+          o[h][e] = ffma2(p2b, make_float2(bf_lo(vwb[e]), bf_hi(vwb[e])), t2);
         }
-        const float p = exp2f(sdot - m[h]);
-        l[h] += p;
-        const float2 pp = make_float2(p, p);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[h][e] = ffma2(pp, make_float2(bf_lo(vw[e]), bf_hi(vw[e])), o[h][e]);
+        m[h] = mn;
       }
     }
   }
@@ -373,19 +421,31 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   const int b = unit / a.Hkv, g = unit % a.Hkv;
   constexpr int PS = part_stride(RG);
   float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * PS;
+  // weights e^(m_w - M) of the 16 warp states and the CTA max / sum, per head
+  float* mw = mer + NWARPS * RG * (kD + 2);   // [NWARPS][RG] weights, then [RG] M, [RG] L
+  if (warp < RG) {
+    const int h = warp;
+    const float mv = lane < NWARPS ? mer[(lane * RG + h) * (kD + 2) + kD] : -INFINITY;
+    float M = mv;
+#pragma unroll
+    for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
+    const float wgt = (lane < NWARPS && M != -INFINITY) ? exp2f(mv - M) : 0.f;
+    float L = lane < NWARPS ? mer[(lane * RG + h) * (kD + 2) + kD + 1] * wgt : 0.f;
+#pragma unroll
+    for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
+    if (lane < NWARPS) mw[lane * RG + h] = wgt;
+    if (lane == 0) {
+      mw[NWARPS * RG + h] = M;
+      mw[NWARPS * RG + RG + h] = L;
+    }
+  }
+  __syncthreads();
   for (int oi = tid; oi < RG * kD; oi += NT) {
     const int h = oi / kD, j = oi % kD;
-    float M = -INFINITY;
-    for (int w = 0; w < NWARPS; ++w) M = fmaxf(M, mer[(w * RG + h) * (kD + 2) + kD]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int w = 0; w < NWARPS; ++w) {
-        const float* src = mer + (w * RG + h) * (kD + 2);
-        const float wgt = exp2f(src[kD] - M);
-        L = fmaf(src[kD + 1], wgt, L);
-        O = fmaf(src[j], wgt, O);
-      }
-    }
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w) O = fmaf(mer[(w * RG + h) * (kD + 2) + j], mw[w * RG + h], O);
+    const float M = mw[NWARPS * RG + h], L = mw[NWARPS * RG + RG + h];
     if (a.C == 1) {
       a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
     } else {
@@ -406,7 +466,6 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   }
   __syncthreads();
   if (!s_int[0]) return;
-  __threadfence();
   if (a.C > 1) {
     // all C partial states of the unit into shared memory in one pass
     const float* parts = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit) * PS;
@@ -416,20 +475,32 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     for (int i = tid; i < n4; i += NT)
       reinterpret_cast<float4*>(sp)[i] = __ldcg(reinterpret_cast<const float4*>(parts) + i);
     __syncthreads();
+    // weights e^(m_c - M) of every CTA's state and 1 / sum, once per head
+    float* sw = sp + a.C * PS;              // [C][RG]
+    float* sinv = sw + a.C * RG;            // [RG]
+    if (warp < RG) {
+      const int h = warp;
+      float M = -INFINITY;
+      for (int cc = lane; cc < a.C; cc += 32) M = fmaxf(M, sp[cc * PS + h * (kD + 2) + kD]);
+#pragma unroll
+      for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
+      float L = 0.f;
+      for (int cc = lane; cc < a.C; cc += 32) {
+        const float* src = sp + cc * PS + h * (kD + 2);
+        const float wgt = (M == -INFINITY) ? 0.f : exp2f(src[kD] - M);
+        sw[cc * RG + h] = wgt;
+        L = fmaf(src[kD + 1], wgt, L);
+      }
+#pragma unroll
+      for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
+      if (lane == 0) sinv[h] = (L > 0.f) ? 1.f / L : 0.f;
+    }
+    __syncthreads();
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
-      float M = -INFINITY;
-      for (int cc = 0; cc < a.C; ++cc) M = fmaxf(M, sp[cc * PS + h * (kD + 2) + kD]);
-      float L = 0.f, O = 0.f;
-      if (M != -INFINITY) {
-        for (int cc = 0; cc < a.C; ++cc) {
-          const float* src = sp + cc * PS + h * (kD + 2);
-          const float wgt = exp2f(src[kD] - M);
-          L = fmaf(src[kD + 1], wgt, L);
-          O = fmaf(src[j], wgt, O);
-        }
-      }
-      a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
+      float O = 0.f;
+      for (int cc = 0; cc < a.C; ++cc) O = fmaf(sp[cc * PS + h * (kD + 2) + j], sw[cc * RG + h], O);
+      a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = O * sinv[h];
     }
   }
   if (tid == 0) atomicExch(a.counters + unit, 0u);
@@ -440,7 +511,7 @@ template <int RG, int WORDS, int MODE>
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_int[NWARPS + 16];
-  __shared__ int s_aux[2 * kMaxCtasPerUnit];
+  __shared__ int s_aux[264];  // distance totals (<= 257 bins)
   __shared__ float s_flt[4];
   constexpr int BITS = WORDS * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -522,15 +593,16 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       const long long wpb = pb + static_cast<long long>(my_pages) * warp / NWARPS;
       const long long wpe = pb + static_cast<long long>(my_pages) * (warp + 1) / NWARPS;
       const int w_pages = static_cast<int>(wpe - wpb);
-      const int n_grp = (w_pages + kPagesPerGroup - 1) / kPagesPerGroup;
+      constexpr int PPG = (RG <= 4) ? 8 : 4;        // pages per warp step (NV = PPG * r <= 32)
+      const int n_grp = (w_pages + PPG - 1) / PPG;
       const uint16_t* meta_u = a.meta + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
       const uint4* wsrc = reinterpret_cast<const uint4*>(meta_u + wpb * 2 * kD) + lane;  // 32 x 16 B per page
       uint4* lslots = reinterpret_cast<uint4*>(S.scratch) + warp * kLaneSlots * 32 + lane;
-      auto issue_group = [&](int gi) {  // every lane: its 16 B of four pages, one commit group
+      auto issue_group = [&](int gi) {  // every lane: its 16 B of PPG pages, one commit group
         if (gi < n_grp) {
 #pragma unroll
-          for (int pp = 0; pp < kPagesPerGroup; ++pp) {
-            const int pg = gi * kPagesPerGroup + pp;
+          for (int pp = 0; pp < PPG; ++pp) {
+            const int pg = gi * PPG + pp;
             if (pg < w_pages) cp_async16(lslots + (pg % kLaneSlots) * 32, wsrc + static_cast<size_t>(pg) * 32);
           }
         }
@@ -542,7 +614,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         bulk_g2s(smem_addr(sRW), Rg, kD * kD * sizeof(float), rw_addr);
       }
 #pragma unroll
-      for (int gi = 0; gi < kLaneSlots / kPagesPerGroup; ++gi) issue_group(gi);
+      for (int gi = 0; gi < kLaneSlots / PPG; ++gi) issue_group(gi);
       if (!wait_rw()) {
         cp_async_wait<0>();
         if (tid == 0) {
@@ -571,7 +643,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       // bounds and hold max(q~, 0), so Eq. 3 is one multiply-add per stored
       // bound.  A stage's four pages x r heads partial sums are folded with a
       // butterfly reduce-scatter, then the max over the heads is taken.
-      constexpr int NV = kPagesPerGroup * RG;
+      constexpr int NV = PPG * RG;
       constexpr int LNV = Log2<NV>::value;
       constexpr int SH = 5 - LNV;                   // lanes sharing one value index
       static_assert(NV <= 32, "at most 32 partial sums per lane");
@@ -588,13 +660,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       float* wsU_u = a.wsU + static_cast<size_t>(unit) * a.np_stride;
       float lmin = INFINITY, lmax = -INFINITY;
       for (int gi = 0; gi < n_grp; ++gi) {
-        cp_async_wait<kLaneSlots / kPagesPerGroup - 1>();   // this lane's group gi has landed
-        const int spages = min(kPagesPerGroup, w_pages - gi * kPagesPerGroup);
+        cp_async_wait<kLaneSlots / PPG - 1>();   // this lane's group gi has landed
+        const int spages = min(PPG, w_pages - gi * PPG);
         float v[NV];
 #pragma unroll
-        for (int pp = 0; pp < kPagesPerGroup; ++pp) {
+        for (int pp = 0; pp < PPG; ++pp) {
           uint4 x = make_uint4(0u, 0u, 0u, 0u);
-          if (pp < spages) x = lslots[((gi * kPagesPerGroup + pp) % kLaneSlots) * 32];
+          if (pp < spages) x = lslots[((gi * PPG + pp) % kLaneSlots) * 32];
           const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
           for (int h = 0; h < RG; ++h) {
@@ -604,7 +676,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
             v[pp * RG + h] = acc.x + acc.y;
           }
         }
-        issue_group(gi + kLaneSlots / kPagesPerGroup);  // refill the slots just read
+        issue_group(gi + kLaneSlots / PPG);  // refill the slots just read
         reduce_scatter<NV>(v, lane);
         const int idx = lane >> SH;
         float u = v[0];
@@ -612,7 +684,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         for (int mm = 1; mm < RG; mm <<= 1) u = fmaxf(u, __shfl_xor_sync(0xFFFFFFFFu, u, mm << SH));
         const int pl = idx / RG;
         if ((idx % RG) == 0 && (lane & ((1 << SH) - 1)) == 0 && pl < spages) {
-          const long long pg = wpb + static_cast<long long>(gi) * kPagesPerGroup + pl;
+          const long long pg = wpb + static_cast<long long>(gi) * PPG + pl;
           wsU_u[pg] = u;
           if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
           lmin = fminf(lmin, u);
@@ -839,28 +911,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
           }
         } else {
           // many equal-looking bounds: exact search for the Pk-th largest key
-          uint32_t T = 0u;
-          for (int bit = 31; bit >= 0; --bit) {
-            const uint32_t cand = T | (1u << bit);
-            int cnt = 0;
-            for (int p = tid; p < NP; p += NT) cnt += order_key(sU[p]) >= cand;
-            if (block_sum(cnt, s_scan) >= Pk) T = cand;
-          }
-          int gt = 0;
-          for (int p = tid; p < NP; p += NT) gt += order_key(sU[p]) > T;
-          const int need_eq = Pk - block_sum(gt, s_scan);
-          const int span = (NP + NT - 1) / NT;
-          const int lo = tid * span, hi = min(NP, lo + span);
-          int eq = 0;
-          for (int p = lo; p < hi; ++p) eq += order_key(sU[p]) == T;
-          int eqtot;
-          int er = block_excl_scan(eq, s_scan, &eqtot);
-          for (int p = lo; p < hi; ++p) {
-            const uint32_t kk = order_key(sU[p]);
-            bool keep = kk > T;
-            if (kk == T) keep = (er++ < need_eq);
-            if (keep) atomicOr(&sBits[p >> 5], 1u << (p & 31));
-          }
+          exact_top_pages(sU, NP, Pk, s_scan, sBits);
         }
       }
       __syncthreads();
@@ -1017,80 +1068,132 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         for (int i = tid; i < a.C * (BITS + 1); i += NT) sHA[i] = __ldcg(hall + i);
       }
       __syncthreads();
-      int tv = 0;
-      if (tid <= BITS)
-        for (int cc = 0; cc < a.C; ++cc) tv += sHA[cc * (BITS + 1) + tid];
-      int n_cand;
-      const int cum = block_excl_scan(tv, s_scan, &n_cand);
-      const int k_eff = min(a.k, n_cand);
-      if (tid == 0) {
-        s_misc[5] = -1;
-        s_misc[6] = 0;
+      // distance totals tot[v] = sum over CTAs (thread v)
+      int* stv = s_aux;                                  // [BITS + 1] <= 257 ints
+      int* sbe = sHA + a.C * (BITS + 1);                 // [C][2]: below T, at T
+      if (tid <= BITS) {
+        int x = 0;
+        for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * (BITS + 1) + tid];
+        stv[tid] = x;
       }
       __syncthreads();
-      if (tid <= BITS && tv > 0 && cum < k_eff && cum + tv >= k_eff) {
-        s_misc[5] = tid;
-        s_misc[6] = k_eff - cum;
-      }
-      __syncthreads();
-      const int T = s_misc[5];
-      const int needT = s_misc[6];
-      int* sBelow = s_aux;
-      int* sEq = s_aux + kMaxCtasPerUnit;
-      for (int cc = warp; cc < a.C; cc += NWARPS) {  // one warp per CTA row
-        int below = 0;
-        for (int v = lane; v < T; v += 32) below += sHA[cc * (BITS + 1) + v];
+      if (warp == 0) {  // threshold T: the k_eff-th smallest distance, and k_eff
+        constexpr int VPL = (BITS + 1 + 31) / 32;
+        int total = 0;
 #pragma unroll
-        for (int o2 = 16; o2 >= 1; o2 >>= 1) below += __shfl_xor_sync(0xFFFFFFFFu, below, o2);
+        for (int kk = 0; kk < VPL; ++kk) total += (lane + 32 * kk <= BITS) ? stv[lane + 32 * kk] : 0;
+#pragma unroll
+        for (int o2 = 16; o2 >= 1; o2 >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o2);
+        const int k_eff = min(a.k, total);
+        int T = -1, run = 0;
+#pragma unroll
+        for (int kk = 0; kk < VPL; ++kk) {
+          const int v = lane + 32 * kk;
+          const int x = v <= BITS ? stv[v] : 0;
+          int incl = x;
+#pragma unroll
+          for (int o2 = 1; o2 < 32; o2 <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
+            if (lane >= o2) incl += y;
+          }
+          const int excl = run + incl - x;
+          const unsigned hit = __ballot_sync(0xFFFFFFFFu, x > 0 && excl < k_eff && excl + x >= k_eff);
+          if (hit && T < 0) {
+            const int src = __ffs(hit) - 1;
+            T = 32 * kk + src;
+            const int need = k_eff - __shfl_sync(0xFFFFFFFFu, excl, src);
+            if (lane == 0) s_misc[4] = need;
+          }
+          run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
         if (lane == 0) {
-          sBelow[cc] = below;
-          sEq[cc] = T >= 0 ? sHA[cc * (BITS + 1) + T] : 0;
+          s_misc[5] = T;
+          s_misc[6] = k_eff;
+          if (T < 0) s_misc[4] = 0;
         }
       }
       __syncthreads();
-      if (tid == 0) {
+      {
+        // per-CTA tokens below T / at T: a half-warp per CTA row
+        const int T = s_misc[5];
+        // warp-uniform trip count: each warp takes rows base and base + 1
+        for (int base = warp * 2; base < a.C; base += NT / 16) {
+          const int cc = base + (lane >> 4), part = lane & 15;
+          const bool row_ok = cc < a.C;
+          int below = 0;
+          if (row_ok)
+            for (int v = part; v < T; v += 16) below += sHA[cc * (BITS + 1) + v];
+#pragma unroll
+          for (int o2 = 8; o2 >= 1; o2 >>= 1) below += __shfl_xor_sync(0xFFFFFFFFu, below, o2);
+          if (row_ok && part == 0) {
+            sbe[2 * cc] = below;
+            sbe[2 * cc + 1] = T >= 0 ? sHA[cc * (BITS + 1) + T] : 0;
+          }
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {  // in CTA order: tie quota and output offset of each CTA
+        const int needT = s_misc[4];
         int pre_eq = 0, off = 0;
-        for (int cc = 0; cc < a.C; ++cc) {
-          const int quota = max(0, min(needT - pre_eq, sEq[cc]));
-          const int selc = sBelow[cc] + quota;
+        for (int c0 = 0; c0 < a.C; c0 += 32) {
+          const int cc = c0 + lane;
+          const int below = cc < a.C ? sbe[2 * cc] : 0;
+          const int eq = cc < a.C ? sbe[2 * cc + 1] : 0;
+          int eq_in = eq;
+#pragma unroll
+          for (int o2 = 1; o2 < 32; o2 <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, eq_in, o2);
+            if (lane >= o2) eq_in += y;
+          }
+          const int quota = max(0, min(needT - (pre_eq + eq_in - eq), eq));
+          const int selc = below + quota;
+          int sel_in = selc;
+#pragma unroll
+          for (int o2 = 1; o2 < 32; o2 <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, sel_in, o2);
+            if (lane >= o2) sel_in += y;
+          }
           if (cc == c) {
-            s_misc[7] = off;
+            s_misc[7] = off + sel_in - selc;
             s_misc[8] = quota;
             s_misc[9] = selc;
           }
-          pre_eq += sEq[cc];
-          off += selc;
+          pre_eq += __shfl_sync(0xFFFFFFFFu, eq_in, 31);
+          off += __shfl_sync(0xFFFFFFFFu, sel_in, 31);
         }
       }
       __syncthreads();
+      const int T = s_misc[5], k_eff = s_misc[6];
       const int my_off = s_misc[7], my_quota = s_misc[8], my_sel = s_misc[9];
       {
+        // one packed scan: (tokens below T) | (tokens at T) << 16
         const int span = (ntok + NT - 1) / NT;
         const int lo = tid * span, hi = min(ntok, lo + span);
-        int eq = 0;
-        for (int i = lo; i < hi; ++i) eq += S.tokD[i] == T;
-        int tmp;
-        const int eq_pre = block_excl_scan(eq, s_scan, &tmp);
-        int er = eq_pre, cnt = 0;
+        int lt = 0, eq = 0;
         for (int i = lo; i < hi; ++i) {
           const int D = S.tokD[i];
-          bool f = D < T;
-          if (D == T) f = (er++ < my_quota);
-          cnt += f;
+          lt += D < T;
+          eq += D == T;
         }
-        int pos = block_excl_scan(cnt, s_scan, &tmp);
-        er = eq_pre;
+        int tmp;
+        const int pre = block_excl_scan(lt | (eq << 16), s_scan, &tmp);
+        int lt_b = pre & 0xFFFF, eq_b = pre >> 16;
         int32_t* tout = a.tok_idx + static_cast<size_t>(unit) * a.k;
         for (int i = lo; i < hi; ++i) {
           const int D = S.tokD[i];
-          bool f = D < T;
-          if (D == T) f = (er++ < my_quota);
-          if (f) {
+          int pos = -1;
+          if (D < T) {
+            pos = lt_b + min(eq_b, my_quota);
+            ++lt_b;
+          } else if (D == T) {
+            if (eq_b < my_quota) pos = lt_b + eq_b;
+            ++eq_b;
+          }
+          if (pos >= 0) {
             const int slot = i / S_;
             const int n = S.my_pages[slot] * S_ + (i - slot * S_);
             tout[my_off + pos] = n;
             S.sel[pos] = n;
-            ++pos;
           }
         }
         if (c == 0) {

@@ -19,7 +19,6 @@ constexpr int kCandMax = 1024;          // boundary-bucket candidates held in sh
 constexpr int kRankDirect = 48;         // at most this many are ranked without a second level
 constexpr int kMaxTokensPerCta = 16384; // candidate tokens one CTA scores
 constexpr int kAttnSlots = 8;           // K/V tokens in flight per half-warp
-constexpr int kPagesPerGroup = 4;      // pages a warp scores per step (one copy group)
 constexpr int kLaneSlots = 16;         // pages in flight per warp (8 KiB)
 constexpr unsigned long long kSpinLimit = 1ull << 31;  // ~1 s at 2 GHz
 
@@ -109,12 +108,12 @@ inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, 
         + sizeof(uint32_t) * align_up(((size_t)NP + 31) / 32, 4)  // kept bitmap
         + 2 * (sizeof(float) + sizeof(int)) * kCandMax       // boundary candidates, 2 levels
         + sizeof(float) * 2 * (kDecodeThreads / 32);          // level-2 min / max
-    hist = sizeof(int) * (size_t)C * (bits + 1) + 16;
+    hist = sizeof(int) * ((size_t)C * (bits + 1) + 2 * (size_t)C) + 16;
   }
   if (mode != kModeSelect) {
     const size_t ring = (size_t)32 * kAttnSlots * 16 * 2 * 16;  // half-warps x slots x lanes x (K, V) x 16 B
-    size_t merge = sizeof(float) * (kDecodeThreads / 32) * (size_t)r * (kD + 2);
-    const size_t parts = sizeof(float) * (size_t)C * part_stride(r);  // final merge
+    size_t merge = sizeof(float) * ((kDecodeThreads / 32) * (size_t)r * (kD + 2) + (kDecodeThreads / 32) * (size_t)r + 2 * (size_t)r);
+    const size_t parts = sizeof(float) * ((size_t)C * part_stride(r) + (size_t)C * r + r);  // final merge
     merge = merge > parts ? merge : parts;
     attn = ring > merge ? ring : merge;
   }
