@@ -213,61 +213,69 @@ __device__ void find_boundary(const int* hist, int need, int* s_warp, int* out) 
   __syncthreads();
 }
 
-// Unit barrier: every CTA of the unit adds one to the counter, then waits
-// until it reaches `target`.  Returns false (and records HHR_ERR_TIMEOUT) if
-// the wait ran out.  All threads of the CTA must call it.
-__device__ bool unit_arrive_wait(uint32_t* ctr, uint32_t target, const DecodeArgs& a,
-                                 int* s_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atom_add_acq_rel(ctr, 1u);
-    int ok = 1;
-    const long long t0 = clock64();
-    while (ld_acquire(ctr) < target) {
-      if (static_cast<unsigned long long>(clock64() - t0) > a.spin_limit) {
-        atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-        ok = 0;
-        break;
-      }
-      __nanosleep(32);
-    }
-    __threadfence();
-    *s_flag = ok;
-  }
-  __syncthreads();
-  return *s_flag != 0;
-}
-
-// Butterfly reduce-scatter of NV per-lane partial sums over the 32 lanes.
-// Afterwards v[0] of lane l holds the full sum of value index l >> (5 - log2 NV).
-template <int NV>
-__device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
-  constexpr int L = (NV >= 32) ? 5 : (NV >= 16) ? 4 : (NV >= 8) ? 3 : (NV >= 4) ? 2 : (NV >= 2) ? 1 : 0;
+// One quarter of x[r][d] . M[d][d] (both float32 in shared memory): thread t
+// returns, for every head h, the sum over rows i in [32 (t / 128), 32 (t / 128) + 32)
+// of x[h][i] * M[i][t % 128].  M is read once per CTA, conflict-free; x by
+// broadcast.  The caller adds the four quarters.
+template <int RG>
+__device__ __forceinline__ void quarter_product(const float* x, const float* M, float (&acc)[RG]) {
+  static_assert(NT == 4 * kD, "four row quarters of 128 columns");
+  const int j = threadIdx.x & (kD - 1), i0 = (threadIdx.x >> 7) * 32;
 #pragma unroll
-  for (int k = 0; k < L; ++k) {
-    const int m = 16 >> k;
-    const int h = NV >> (k + 1);
-    const bool up = (lane & m) != 0;
+  for (int h = 0; h < RG; ++h) acc[h] = 0.f;
+#pragma unroll 2
+  for (int ii = 0; ii < 32; ii += 4) {
+    float m[4];
 #pragma unroll
-    for (int i = 0; i < h; ++i) {
-      const float send = up ? v[i] : v[i + h];
-      const float keep = up ? v[i + h] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, m);
+    for (int e = 0; e < 4; ++e) m[e] = M[(i0 + ii + e) * kD + j];
+#pragma unroll
+    for (int h = 0; h < RG; ++h) {
+      const float4 xv = *reinterpret_cast<const float4*>(x + h * kD + i0 + ii);
+      acc[h] = fmaf(xv.x, m[0], acc[h]);
+      acc[h] = fmaf(xv.y, m[1], acc[h]);
+      acc[h] = fmaf(xv.z, m[2], acc[h]);
+      acc[h] = fmaf(xv.w, m[3], acc[h]);
     }
   }
-#pragma unroll
-  for (int k = L; k < 5; ++k) v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], 16 >> k);
 }
 
-template <int NV>
-struct Log2 {
-  static constexpr int value = (NV >= 32) ? 5 : (NV >= 16) ? 4 : (NV >= 8) ? 3 : (NV >= 4) ? 2 : (NV >= 2) ? 1 : 0;
-};
+// ldmatrix: four (two) 8x8 b16 matrices; lane i supplies the row address of
+// matrix i / 8, row i % 8 (lanes 0-15 for x2).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
+}
 
+// d += A (16 x 16, row-major bf16) * B (16 x 8, column-major bf16), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+               "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// v = hi + mid + lo exactly, each term a bf16 (v - hi and the next residual
+// are exact in float32, and the last residual has at most 8 significant
+// bits).  Stores the terms at column k of rows n0, n0 + 1, n0 + 2 of the
+// [rows][256] bf16 operand whose 16-B chunks are swizzled by row & 7.
+__device__ __forceinline__ void put_terms(uint16_t* qb, int n0, int k, float v) {
+  float rest = v;
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    const __nv_bfloat16 term = __float2bfloat16_rn(rest);
+    rest -= __bfloat162float(term);
+    const int n = n0 + t;
+    qb[n * (2 * kD) + (((k >> 3) ^ (n & 7)) << 3) + (k & 7)] = __bfloat16_as_ushort(term);
+  }
+}
 
 struct Smem {
-  float* qt;       // [r][d] rotated queries
+  uint16_t* qb;    // bf16 terms of [min(q~, 0) ; max(q~, 0)], [8 nb][2 d], 16-B chunks swizzled
   float* qf;       // [r][d] queries (float), pre-scaled for attention
   uint32_t* qc;    // [r][w] query codes
   int* my_pages;   // kept pages of this CTA's slice
@@ -471,7 +479,7 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     const float* parts = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit) * PS;
     float* sp = reinterpret_cast<float*>(scratch);
     const int n4 = a.C * PS / 4;
-#pragma unroll 4
+#pragma unroll 8
     for (int i = tid; i < n4; i += NT)
       reinterpret_cast<float4*>(sp)[i] = __ldcg(reinterpret_cast<const float4*>(parts) + i);
     __syncthreads();
@@ -518,7 +526,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
   const int c = blockIdx.x % a.C;
   const DecodeSmem lay = decode_smem(a.NP, a.C, BITS, RG, a.slice_pages, a.slice_tokens, MODE);
   Smem S;
-  S.qt = reinterpret_cast<float*>(smem + lay.qt);
+  S.qb = reinterpret_cast<uint16_t*>(smem + lay.qb);
   S.qf = reinterpret_cast<float*>(smem + lay.qf);
   S.qc = reinterpret_cast<uint32_t*>(smem + lay.qc);
   S.my_pages = reinterpret_cast<int*>(smem + lay.my_pages);
@@ -534,18 +542,21 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
     mbar_init(rw_addr, 1u);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if constexpr (MODE != kModeAttend) {
+    // the B operand's unused columns (fourth term of each head, absent heads) stay zero
+    for (int i = tid; i < 8 * ((RG * 4 + 7) / 8) * 2 * kD; i += NT) S.qb[i] = 0;
+  }
   __syncthreads();
 
   for (int unit = blockIdx.x / a.C; unit < a.units; unit += a.grid_units) {
     const int b = unit / a.Hkv, g = unit % a.Hkv;
     uint32_t* ctr = a.counters + unit;
 
-    // queries of the group, as float (raw) -- q~ is derived from these
     const uint16_t* qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * RG) * kD;
-    for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
-    __syncthreads();
 
     if constexpr (MODE == kModeAttend) {
+      for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
+      __syncthreads();
       const int n = a.nsel_in[unit];
       const int s0 = static_cast<int>(static_cast<long long>(c) * n / a.C);
       const int s1 = static_cast<int>(static_cast<long long>(c + 1) * n / a.C);
@@ -560,9 +571,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       continue;
     } else {
       // ---------------------------------------------------------- phase 0
-      // R (and later W) reach shared memory by one bulk copy on their own
-      // mbarrier, requested before any metadata so that q~ = q R is ready
-      // first.  Each warp then streams its own slice of pages.
+      // R reaches shared memory by one bulk copy on its mbarrier, requested
+      // before any metadata.  Every warp streams its own run of pages into a
+      // lane-private ring: the first kLaneSlots pages of each warp at once,
+      // the rest of the ring -- which shares its storage with R -- as soon
+      // as q~ = q R is formed.
       const long long pb = static_cast<long long>(c) * a.NP / a.C;
       const long long pe = static_cast<long long>(c + 1) * a.NP / a.C;
       const int my_pages = static_cast<int>(pe - pb);
@@ -570,6 +583,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       const float* Rg = a.R + static_cast<size_t>(g) * kD * kD;
       const float* Wg = a.W + static_cast<size_t>(g) * kD * BITS;
       auto issue_w = [&](int half_w) {  // thread 0 only: 128 columns of W
+        // the storage was last touched by generic-proxy copies and loads
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
         if constexpr (BITS == kD) {
           bulk_g2s(smem_addr(sRW), Wg, kD * kD * sizeof(float), rw_addr);
@@ -589,21 +604,33 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       // This warp's pages [wpb, wpe).  Lane l only ever reads bytes
       // [16 l, 16 l + 16) of a page, so it copies exactly those bytes into its
       // own shared-memory slots with cp.async and waits on its own copies: no
-      // barrier is involved.  kLaneSlots pages are in flight per warp.
+      // barrier is involved.  Slot s of warp w is the 512 B at
+      // (s * NWARPS + w) * 512: slots [0, kLaneSlots) lie below the R / W
+      // buffer, slots [kLaneSlots, kRingSlots) inside it.
       const long long wpb = pb + static_cast<long long>(my_pages) * warp / NWARPS;
       const long long wpe = pb + static_cast<long long>(my_pages) * (warp + 1) / NWARPS;
       const int w_pages = static_cast<int>(wpe - wpb);
-      constexpr int PPG = (RG <= 4) ? 8 : 4;        // pages per warp step (NV = PPG * r <= 32)
+      constexpr int PPG = 8;                        // pages per ring group; an A tile is two groups
+      constexpr int G0 = kLaneSlots / PPG;          // groups in flight while q~ is formed
+      constexpr int GR = kRingSlots / PPG;          // groups in flight afterwards
+      static_assert(kLaneSlots % PPG == 0 && kRingSlots % PPG == 0, "whole groups per ring");
+      static_assert(GR == 3, "tile ti reads groups 2 ti, 2 ti + 1 and refills them with 2 ti + 3, 2 ti + 4");
+      static_assert((kRingSlots - kLaneSlots) * NWARPS * 512 == kD * kD * sizeof(float),
+                    "the upper ring slots fill the R / W buffer exactly");
       const int n_grp = (w_pages + PPG - 1) / PPG;
       const uint16_t* meta_u = a.meta + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
       const uint4* wsrc = reinterpret_cast<const uint4*>(meta_u + wpb * 2 * kD) + lane;  // 32 x 16 B per page
-      uint4* lslots = reinterpret_cast<uint4*>(S.scratch) + warp * kLaneSlots * 32 + lane;
+      // Within a slot, 16-B chunk c sits at position c ^ (s & 7), so that the
+      // same chunk of 8 consecutive slots covers all banks (ldmatrix below).
+      uint4* ring = reinterpret_cast<uint4*>(S.scratch) + warp * 32;
       auto issue_group = [&](int gi) {  // every lane: its 16 B of PPG pages, one commit group
         if (gi < n_grp) {
 #pragma unroll
           for (int pp = 0; pp < PPG; ++pp) {
             const int pg = gi * PPG + pp;
-            if (pg < w_pages) cp_async16(lslots + (pg % kLaneSlots) * 32, wsrc + static_cast<size_t>(pg) * 32);
+            const int s = pg % kRingSlots;
+            if (pg < w_pages)
+              cp_async16(ring + s * (NWARPS * 32) + (lane ^ (s & 7)), wsrc + static_cast<size_t>(pg) * 32);
           }
         }
         cp_async_commit();
@@ -614,7 +641,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         bulk_g2s(smem_addr(sRW), Rg, kD * kD * sizeof(float), rw_addr);
       }
 #pragma unroll
-      for (int gi = 0; gi < kLaneSlots / PPG; ++gi) issue_group(gi);
+      for (int gi = 0; gi < G0; ++gi) issue_group(gi);
+      // queries of the group, as float (raw) -- q~ is derived from these
+      for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
       if (!wait_rw()) {
         cp_async_wait<0>();
         if (tid == 0) {
@@ -624,112 +653,118 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         __syncthreads();
         return;
       }
-      for (int oi = tid; oi < RG * kD; oi += NT) {
-        const int h = oi / kD, j = oi % kD;
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 8
-        for (int i = 0; i < kD; i += 2)
-          acc = ffma2(make_float2(S.qf[h * kD + i], S.qf[h * kD + i + 1]),
-                      make_float2(sRW[i * kD + j], sRW[(i + 1) * kD + j]), acc);
-        S.qt[oi] = acc.x + acc.y;
+      {
+        float acc[RG];
+        quarter_product<RG>(S.qf, sRW, acc);
+        __syncthreads();                            // every thread has read R
+        float* part = sRW;                          // [4][r][d] quarter sums, over R
+#pragma unroll
+        for (int h = 0; h < RG; ++h) part[((tid >> 7) * RG + h) * kD + (tid & (kD - 1))] = acc[h];
+        __syncthreads();
+        for (int oi = tid; oi < RG * kD; oi += NT) {
+          const float qt = (part[oi] + part[RG * kD + oi]) + (part[2 * RG * kD + oi] + part[3 * RG * kD + oi]);
+          const int h = oi / kD, j = oi % kD;
+          put_terms(S.qb, 4 * h, j, fminf(qt, 0.f));
+          put_terms(S.qb, 4 * h, kD + j, fmaxf(qt, 0.f));
+        }
+        __syncthreads();
       }
-      __syncthreads();
-      // the first 128 columns of W stream in while the page bounds run
-      if (tid == 0) issue_w(0);
+      // the upper ring slots now own the R / W storage
+#pragma unroll
+      for (int gi = G0; gi < GR; ++gi) issue_group(gi);
 
       // ---------------------------------------------------------- phase 1
-      // Warp-per-page scoring.  A 512-B page is one 16-B load per lane: lanes
-      // 0-15 read lower bounds and hold min(q~, 0), lanes 16-31 read upper
-      // bounds and hold max(q~, 0), so Eq. 3 is one multiply-add per stored
-      // bound.  A stage's four pages x r heads partial sums are folded with a
-      // butterfly reduce-scatter, then the max over the heads is taken.
-      constexpr int NV = PPG * RG;
-      constexpr int LNV = Log2<NV>::value;
-      constexpr int SH = 5 - LNV;                   // lanes sharing one value index
-      static_assert(NV <= 32, "at most 32 partial sums per lane");
-      const int half = lane >> 4, dl = (lane & 15) * 8;
-      float2 qs[RG][4];
-#pragma unroll
-      for (int h = 0; h < RG; ++h)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float v0 = S.qt[h * kD + dl + 2 * e], v1 = S.qt[h * kD + dl + 2 * e + 1];
-          qs[h][e] = half ? make_float2(fmaxf(v0, 0.f), fmaxf(v1, 0.f))
-                          : make_float2(fminf(v0, 0.f), fminf(v1, 0.f));
-        }
+      // Eq. 3 as a contraction: with b_h = [min(q~_h, 0) ; max(q~_h, 0)] and a
+      // page's stored bounds [l ; u] (256 bf16), U_p = max_h [l ; u] . b_h.
+      // Each warp multiplies tiles of 16 of its pages -- A fragments loaded
+      // by ldmatrix straight from its ring -- by B = the exact bf16 terms of
+      // the b_h (4 columns per head) on the tensor cores, fp32 accumulation.
+      constexpr int NB = (RG * 4 + 7) / 8;          // n8 column blocks of B
       float* wsU_u = a.wsU + static_cast<size_t>(unit) * a.np_stride;
       float lmin = INFINITY, lmax = -INFINITY;
-      for (int gi = 0; gi < n_grp; ++gi) {
-        cp_async_wait<kLaneSlots / PPG - 1>();   // this lane's group gi has landed
-        const int spages = min(PPG, w_pages - gi * PPG);
-        float v[NV];
+      const int n_tiles = (w_pages + 15) / 16;
+      const int lm = lane >> 3, lr = lane & 7;      // ldmatrix: matrix, row
+      const int g8 = lane >> 2, t4 = lane & 3;      // mma fragment: row, column pair
+      const uint32_t ring_s = smem_addr(S.scratch) + warp * 512;
+      const uint32_t qb_s = smem_addr(S.qb);
+      for (int ti = 0; ti < n_tiles; ++ti) {
+        cp_async_wait<1>();   // this lane's groups 2 ti and 2 ti + 1 have landed
+        __syncwarp();         // ... and every lane's
+        // A row (lm & 1) * 8 + lr of the tile is page 16 ti + that row
+        const uint32_t a_row = ring_s + (((2 * ti + (lm & 1)) % GR) * PPG + lr) * (NWARPS * 512);
+        float acc[NB][4];
 #pragma unroll
-        for (int pp = 0; pp < PPG; ++pp) {
-          uint4 x = make_uint4(0u, 0u, 0u, 0u);
-          if (pp < spages) x = lslots[((gi * PPG + pp) % kLaneSlots) * 32];
-          const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-          for (int h = 0; h < RG; ++h) {
-            float2 acc = make_float2(0.f, 0.f);
+          for (int e = 0; e < 4; ++e) acc[nb][e] = 0.f;
+#pragma unroll 4
+        for (int ks = 0; ks < 2 * kD / 16; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a_row + (static_cast<uint32_t>((2 * ks + (lm >> 1)) ^ lr) << 4), a0, a1, a2, a3);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc = ffma2(qs[h][e], make_float2(bf_lo(xw[e]), bf_hi(xw[e])), acc);
-            v[pp * RG + h] = acc.x + acc.y;
+          for (int nb = 0; nb < NB; nb += 2) {
+            if (nb + 1 < NB) {
+              uint32_t b0, b1, b2, b3;
+              const int n = (nb + (lm >> 1)) * 8 + lr;
+              ldsm_x4(qb_s + n * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1, b2, b3);
+              mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
+              mma_bf16_16816(acc[nb + 1], a0, a1, a2, a3, b2, b3);
+            } else {
+              uint32_t b0, b1;
+              ldsm_x2(qb_s + (nb * 8 + lr) * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1);
+              mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
+            }
           }
         }
-        issue_group(gi + kLaneSlots / PPG);  // refill the slots just read
-        reduce_scatter<NV>(v, lane);
-        const int idx = lane >> SH;
-        float u = v[0];
+        __syncwarp();
+        issue_group(2 * ti + GR);       // refill the slots just read
+        issue_group(2 * ti + GR + 1);
+        // lane (g8, t4) holds columns 8 nb + 2 t4, + 1 (head 2 nb + t4 / 2)
+        // of tile rows g8 and g8 + 8: add the terms, then take the max over
+        // the heads
+        float u0 = -INFINITY, u1 = -INFINITY;
 #pragma unroll
-        for (int mm = 1; mm < RG; mm <<= 1) u = fmaxf(u, __shfl_xor_sync(0xFFFFFFFFu, u, mm << SH));
-        const int pl = idx / RG;
-        if ((idx % RG) == 0 && (lane & ((1 << SH) - 1)) == 0 && pl < spages) {
-          const long long pg = wpb + static_cast<long long>(gi) * PPG + pl;
-          wsU_u[pg] = u;
-          if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
-          lmin = fminf(lmin, u);
-          lmax = fmaxf(lmax, u);
+        for (int nb = 0; nb < NB; ++nb) {
+          float s0 = acc[nb][0] + acc[nb][1];
+          float s1 = acc[nb][2] + acc[nb][3];
+          s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
+          s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
+          if (2 * nb + (t4 >> 1) >= RG) {
+            s0 = -INFINITY;
+            s1 = -INFINITY;
+          }
+          u0 = fmaxf(u0, fmaxf(s0, __shfl_xor_sync(0xFFFFFFFFu, s0, 2)));
+          u1 = fmaxf(u1, fmaxf(s1, __shfl_xor_sync(0xFFFFFFFFu, s1, 2)));
+        }
+        if (t4 == 0) {
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const int pl = ti * 16 + g8 + 8 * hr;
+            if (pl < w_pages) {
+              const float u = hr ? u1 : u0;
+              const long long pg = wpb + pl;
+              wsU_u[pg] = u;
+              if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
+              lmin = fminf(lmin, u);
+              lmax = fmaxf(lmax, u);
+            }
+          }
         }
       }
       cp_async_wait<0>();
-      // query codes (Eq. 10 + sign) from W in shared memory, 128 columns at
-      // a time
-      int w_done = 0;
-      bool q_ok = true;
-      while (q_ok && w_done < BITS / kD) {
-        q_ok = wait_rw();
-        if (!q_ok) break;
-        for (int oi = tid; oi < RG * kD; oi += NT) {  // warp-uniform trip count
-          const int h = oi / kD, t = oi % kD;
-          float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 8
-          for (int i = 0; i < kD; i += 2)
-            acc = ffma2(make_float2(S.qf[h * kD + i], S.qf[h * kD + i + 1]),
-                        make_float2(sRW[i * kD + t], sRW[(i + 1) * kD + t]), acc);
-          const uint32_t word = __ballot_sync(0xFFFFFFFFu, acc.x + acc.y > 0.f);
-          if (lane == 0) S.qc[h * WORDS + w_done * (kD / 32) + t / 32] = word;
-        }
-        ++w_done;
-        if (w_done < BITS / kD) {
-          __syncthreads();
-          if (tid == 0) issue_w(w_done);
-        }
-      }
-      if (__syncthreads_or(!q_ok)) {
-        if (tid == 0) atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-        return;
-      }
       // CTA min / max of its bounds
 #pragma unroll
       for (int o2 = 16; o2 >= 1; o2 >>= 1) {
         lmin = fminf(lmin, __shfl_xor_sync(0xFFFFFFFFu, lmin, o2));
         lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o2));
       }
-      float* red = reinterpret_cast<float*>(S.scratch);
+      float* red = reinterpret_cast<float*>(s_aux);
       if (lane == 0) {
         red[warp] = lmin;
         red[NWARPS + warp] = lmax;
       }
+      // every lane's ring copies have landed and been read: the R / W
+      // storage is free for W
       __syncthreads();
       if (tid == 0) {
         float mn = INFINITY, mx = -INFINITY;
@@ -740,13 +775,41 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         float* mm2 = a.wsMinMax + 2 * static_cast<size_t>(unit * kMaxCtasPerUnit + c);
         mm2[0] = mn;
         mm2[1] = mx;
-      }
-
-      // unit barrier 1; the query codes are computed while waiting
-      __syncthreads();
-      if (tid == 0) {
+        issue_w(0);
+        // unit barrier 1: arrive now, wait after the query codes
         __threadfence();
         atom_add_acq_rel(ctr, 1u);
+      }
+      // query codes (Eq. 10 + sign) from W in shared memory, 128 columns at
+      // a time, while the other CTAs of the unit finish their bounds
+      int w_done = 0;
+      bool q_ok = true;
+      while (w_done < BITS / kD) {
+        q_ok = wait_rw();
+        if (!q_ok) break;
+        float acc[RG];
+        quarter_product<RG>(S.qf, sRW, acc);
+        float* part = reinterpret_cast<float*>(S.scratch);  // [4][r][d], in the drained ring
+#pragma unroll
+        for (int h = 0; h < RG; ++h) part[((tid >> 7) * RG + h) * kD + (tid & (kD - 1))] = acc[h];
+        __syncthreads();                            // partial sums visible, this W half read
+        if (w_done + 1 < BITS / kD && tid == 0) issue_w(w_done + 1);
+        for (int oi = tid; oi < RG * kD; oi += NT) {  // warp-uniform trip count
+          const float z = (part[oi] + part[RG * kD + oi]) + (part[2 * RG * kD + oi] + part[3 * RG * kD + oi]);
+          const uint32_t word = __ballot_sync(0xFFFFFFFFu, z > 0.f);
+          const int h = oi / kD, t = oi % kD;
+          if (lane == 0) S.qc[h * WORDS + w_done * (kD / 32) + t / 32] = word;
+        }
+        ++w_done;
+        if (w_done < BITS / kD) __syncthreads();    // part is rewritten next
+      }
+      if (__syncthreads_or(!q_ok)) {
+        if (tid == 0) {
+          atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+          mbar_wait(rw_addr, (rw_seq - 1) & 1u, a.spin_limit);   // a copy may still be in flight
+        }
+        __syncthreads();
+        return;
       }
       if (tid == 0) {
         int ok = 1;

@@ -19,7 +19,8 @@ constexpr int kCandMax = 1024;          // boundary-bucket candidates held in sh
 constexpr int kRankDirect = 48;         // at most this many are ranked without a second level
 constexpr int kMaxTokensPerCta = 16384; // candidate tokens one CTA scores
 constexpr int kAttnSlots = 8;           // K/V tokens in flight per half-warp
-constexpr int kLaneSlots = 16;         // pages in flight per warp (8 KiB)
+constexpr int kLaneSlots = 16;         // ring slots per warp below the R / W buffer (8 KiB)
+constexpr int kRingSlots = 24;         // ring slots per warp in all (12 KiB), the upper 8 over R / W
 constexpr unsigned long long kSpinLimit = 1ull << 31;  // ~1 s at 2 GHz
 
 inline __host__ __device__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -95,14 +96,14 @@ struct EncodeArgs {
 
 // Shared-memory bytes of a decode CTA (host and device agree on the carve-up).
 struct DecodeSmem {
-  size_t qt, qf, qc, my_pages, tokD, sel, scratch, total;
+  size_t qb, qf, qc, my_pages, tokD, sel, scratch, total;
 };
 
 inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, int r, int mode) {
   size_t sel = 0, hist = 0, attn = 0, stream = 0;
   if (mode != kModeAttend) {
-    // per-warp metadata rings + R / W staging (phases 0-1)
-    stream = (size_t)(kDecodeThreads / 32) * kLaneSlots * 512 + sizeof(float) * kD * kD;
+    // per-warp metadata rings; their upper slots double as R / W staging
+    stream = (size_t)(kDecodeThreads / 32) * kRingSlots * 512;
     sel = sizeof(float) * align_up((size_t)NP, 4)          // U of every page
         + sizeof(int) * kBuckets                             // histogram
         + sizeof(uint32_t) * align_up(((size_t)NP + 31) / 32, 4)  // kept bitmap
@@ -126,7 +127,7 @@ inline __host__ __device__ DecodeSmem decode_smem(int NP, int C, int bits, int r
                                                   int slice_tokens, int mode) {
   DecodeSmem s;
   size_t off = 0;
-  s.qt = off;       off += align_up(sizeof(float) * r * kD, 16);
+  s.qb = off;       off += (size_t)8 * ((r * 4 + 7) / 8) * 2 * kD * 2;  // bf16 terms of q~, [8 nb][2 d]
   s.qf = off;       off += align_up(sizeof(float) * r * kD, 16);
   s.qc = off;       off += align_up(sizeof(uint32_t) * r * (bits / 32), 16);
   s.my_pages = off; off += align_up(sizeof(int) * (size_t)(slice_pages + 1), 16);
