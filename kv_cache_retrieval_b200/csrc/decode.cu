@@ -88,11 +88,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
-// Brings the 128-B line holding `p` into L2 (no register result).
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
-}
-
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
@@ -468,7 +463,6 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   // last CTA of the unit merges the C partial states and resets the counter
   __syncthreads();
   if (tid == 0) {
-    __threadfence();
     const uint32_t old = atom_add_acq_rel(a.counters + unit, 1u);
     s_int[0] = (old == final_target - 1) ? 1 : 0;
   }
@@ -507,6 +501,7 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
       float O = 0.f;
+#pragma unroll 6
       for (int cc = 0; cc < a.C; ++cc) O = fmaf(sp[cc * PS + h * (kD + 2) + j], sw[cc * RG + h], O);
       a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = O * sinv[h];
     }
@@ -766,18 +761,24 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       // every lane's ring copies have landed and been read: the R / W
       // storage is free for W
       __syncthreads();
-      if (tid == 0) {
-        float mn = INFINITY, mx = -INFINITY;
-        for (int w = 0; w < NWARPS; ++w) {
-          mn = fminf(mn, red[w]);
-          mx = fmaxf(mx, red[NWARPS + w]);
+      if (warp == 0) {
+        float mn = lane < NWARPS ? red[lane] : INFINITY;
+        float mx = lane < NWARPS ? red[NWARPS + lane] : -INFINITY;
+#pragma unroll
+        for (int o2 = NWARPS / 2; o2 >= 1; o2 >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o2));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o2));
         }
-        float* mm2 = a.wsMinMax + 2 * static_cast<size_t>(unit * kMaxCtasPerUnit + c);
-        mm2[0] = mn;
-        mm2[1] = mx;
+        if (lane == 0) {
+          float* mm2 = a.wsMinMax + 2 * static_cast<size_t>(unit * kMaxCtasPerUnit + c);
+          mm2[0] = mn;
+          mm2[1] = mx;
+        }
+      }
+      if (tid == 0) {
         issue_w(0);
-        // unit barrier 1: arrive now, wait after the query codes
-        __threadfence();
+        // unit barrier 1: arrive now (the release covers the CTA's U through
+        // the CTA barrier above), wait after the query codes
         atom_add_acq_rel(ctr, 1u);
       }
       // query codes (Eq. 10 + sign) from W in shared memory, 128 columns at
@@ -811,6 +812,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         __syncthreads();
         return;
       }
+      if constexpr (MODE == kModeFused) {
+        // the raw queries have served q~ and the codes: pre-scale them for
+        // attention while the unit barrier completes
+        for (int i = tid; i < RG * kD; i += NT) S.qf[i] *= a.scale_log2;
+      }
       if (tid == 0) {
         int ok = 1;
         const long long t0 = clock64();
@@ -822,7 +828,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
           }
           __nanosleep(32);
         }
-        __threadfence();
         s_misc[0] = ok;
       }
       __syncthreads();
@@ -838,11 +843,18 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       int* sCP = reinterpret_cast<int*>(sCU + kCandMax);
       float* sC2U = reinterpret_cast<float*>(sCP + kCandMax);
       int* sC2P = reinterpret_cast<int*>(sC2U + kCandMax);
+      // all U of the unit, float4 per thread, kept in registers for the
+      // histogram (the tail of a ragged NP goes straight to shared memory)
+      constexpr int kU4 = (HHR_MAX_PAGES / 4 + NT - 1) / NT;
+      const int n4 = NP / 4;
+      float4 ureg[kU4];
       {
-        const int n4 = NP / 4;
         const float4* src4 = reinterpret_cast<const float4*>(wsU_u);
-#pragma unroll 4
-        for (int i = tid; i < n4; i += NT) reinterpret_cast<float4*>(sU)[i] = __ldcg(src4 + i);
+#pragma unroll
+        for (int u = 0; u < kU4; ++u) {
+          const int i = tid + u * NT;
+          ureg[u] = i < n4 ? __ldcg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         for (int p = n4 * 4 + tid; p < NP; p += NT) sU[p] = __ldcg(wsU_u + p);
       }
       for (int i = tid; i < kBuckets; i += NT) sHist[i] = 0;
@@ -866,6 +878,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       }
       if (tid == 0) s_misc[2] = 0;
       __syncthreads();
+#pragma unroll
+      for (int u = 0; u < kU4; ++u) {
+        const int i = tid + u * NT;
+        if (i < n4) reinterpret_cast<float4*>(sU)[i] = ureg[u];
+      }
 
       if (Pk >= NP) {
         for (int p0 = warp * 32; p0 < NP; p0 += NT) {
@@ -880,28 +897,57 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
           const int bk = static_cast<int>((u - gmin) * inv);
           return bk < kBuckets - 1 ? bk : kBuckets - 1;
         };
-        for (int p = tid; p < NP; p += NT) atomicAdd(&sHist[bucket(sU[p])], 1);
+#pragma unroll
+        for (int u = 0; u < kU4; ++u) {
+          if (tid + u * NT < n4) {
+            const int b0 = bucket(ureg[u].x), b1 = bucket(ureg[u].y);
+            const int b2 = bucket(ureg[u].z), b3 = bucket(ureg[u].w);
+            atomicAdd(&sHist[b0], 1);
+            atomicAdd(&sHist[b1], 1);
+            atomicAdd(&sHist[b2], 1);
+            atomicAdd(&sHist[b3], 1);
+          }
+        }
+        for (int p = n4 * 4 + tid; p < NP; p += NT) atomicAdd(&sHist[bucket(sU[p])], 1);
         __syncthreads();
         find_boundary(sHist, Pk, s_scan, &s_misc[3]);
         const int bstar = s_misc[3];
         const int need = Pk - s_misc[4];
         const int cntB = sHist[bstar];
+        // four bitmap words per warp step (independent chains)
         if (cntB == need) {
-          for (int p0 = warp * 32; p0 < NP; p0 += NT) {
-            const int p = p0 + lane;
-            const unsigned word = __ballot_sync(0xFFFFFFFFu, p < NP && bucket(sU[p]) >= bstar);
-            if (lane == 0) sBits[p0 >> 5] = word;
+          for (int p0 = warp * 32; p0 < NP; p0 += 4 * NT) {
+            bool keep[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int p = p0 + u * NT + lane;
+              keep[u] = p < NP && bucket(sU[p]) >= bstar;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int pw = p0 + u * NT;  // warp-uniform
+              const unsigned word = __ballot_sync(0xFFFFFFFFu, keep[u]);
+              if (lane == 0 && pw < NP) sBits[pw >> 5] = word;
+            }
           }
         } else if (cntB <= kCandMax) {
-          for (int p0 = warp * 32; p0 < NP; p0 += NT) {
-            const int p = p0 + lane;
-            const int bk = p < NP ? bucket(sU[p]) : -1;
-            const unsigned word = __ballot_sync(0xFFFFFFFFu, bk > bstar);
-            if (lane == 0) sBits[p0 >> 5] = word;
-            if (bk == bstar) {
-              const int slot = atomicAdd(&s_misc[2], 1);
-              sCU[slot] = sU[p];
-              sCP[slot] = p;
+          for (int p0 = warp * 32; p0 < NP; p0 += 4 * NT) {
+            int bk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int p = p0 + u * NT + lane;
+              bk[u] = p < NP ? bucket(sU[p]) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int pw = p0 + u * NT;  // warp-uniform
+              const unsigned word = __ballot_sync(0xFFFFFFFFu, bk[u] > bstar);
+              if (lane == 0 && pw < NP) sBits[pw >> 5] = word;
+              if (bk[u] == bstar) {
+                const int slot = atomicAdd(&s_misc[2], 1);
+                sCU[slot] = sU[pw + lane];
+                sCP[slot] = pw + lane;
+              }
             }
           }
           __syncthreads();
@@ -966,6 +1012,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
             const float u = fu[i];
             const int pi = fp[i];
             int rank = 0;
+#pragma unroll 8
             for (int j = 0; j < nc; ++j) {
               const float uj = fu[j];
               rank += (uj > u) || (uj == u && fp[j] < pi);
@@ -1061,51 +1108,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         int32_t* hrow = a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * (BITS + 1);
         for (int i = tid; i <= BITS; i += NT) hrow[i] = sHD[i];
       }
-      // unit barrier 2.  While waiting, a fused step prefetches into L2 the
-      // K/V rows of the tokens it most likely keeps: those at or below the
-      // local distance quantile k / (kept tokens), the fraction the global
-      // threshold keeps.  Prefetching changes no result.
+      // unit barrier 2 (the release by thread 0 covers the CTA's histogram
+      // row through the CTA barrier)
       __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        atom_add_acq_rel(ctr, 1u);
-      }
-      if constexpr (MODE == kModeFused) {
-        if (warp == 0) {
-          int local = 0;
-          for (int v = lane; v <= BITS; v += 32) local += sHD[v];
-#pragma unroll
-          for (int o2 = 16; o2 >= 1; o2 >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, o2);
-          const long long cand = static_cast<long long>(Pk) * S_;
-          const long long target = cand > 0 ? (static_cast<long long>(local) * a.k + cand - 1) / cand : 0;
-          int t_loc = -1, run = 0;
-          for (int v0 = 0; v0 <= BITS && t_loc < 0; v0 += 32) {
-            int x = (v0 + lane <= BITS) ? sHD[v0 + lane] : 0;
-#pragma unroll
-            for (int o2 = 1; o2 < 32; o2 <<= 1) {
-              const int y = __shfl_up_sync(0xFFFFFFFFu, x, o2);
-              if (lane >= o2) x += y;
-            }
-            const unsigned hit = __ballot_sync(0xFFFFFFFFu, run + x >= target && target > 0);
-            if (hit) t_loc = v0 + __ffs(hit) - 1;
-            run += __shfl_sync(0xFFFFFFFFu, x, 31);
-          }
-          if (lane == 0) s_misc[10] = (target >= local) ? BITS : t_loc;
-        }
-        __syncthreads();
-        const int t_loc = s_misc[10];
-        const size_t unit_rows = static_cast<size_t>(unit) * a.n_cap;
-        for (int i = tid; i < ntok; i += NT) {
-          if (static_cast<int>(S.tokD[i]) <= t_loc) {
-            const int slot = i / S_;
-            const size_t n = static_cast<size_t>(S.my_pages[slot]) * S_ + (i - slot * S_);
-            prefetch_l2(a.K + (unit_rows + n) * kD);
-            prefetch_l2(a.K + (unit_rows + n) * kD + 64);
-            prefetch_l2(a.V + (unit_rows + n) * kD);
-            prefetch_l2(a.V + (unit_rows + n) * kD + 64);
-          }
-        }
-      }
+      if (tid == 0) atom_add_acq_rel(ctr, 1u);
       if (tid == 0) {
         int ok = 1;
         const long long t0 = clock64();
@@ -1117,7 +1123,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
           }
           __nanosleep(32);
         }
-        __threadfence();
         s_misc[0] = ok;
       }
       __syncthreads();
@@ -1131,49 +1136,28 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         for (int i = tid; i < a.C * (BITS + 1); i += NT) sHA[i] = __ldcg(hall + i);
       }
       __syncthreads();
-      // distance totals tot[v] = sum over CTAs (thread v)
-      int* stv = s_aux;                                  // [BITS + 1] <= 257 ints
+      // distance totals tot[v] = sum over the CTAs (thread v); one block-wide
+      // exclusive scan of them gives k_eff, the threshold distance T (the
+      // k_eff-th smallest) and how many tokens at T are still needed
       int* sbe = sHA + a.C * (BITS + 1);                 // [C][2]: below T, at T
-      if (tid <= BITS) {
-        int x = 0;
-        for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * (BITS + 1) + tid];
-        stv[tid] = x;
+      if (tid == 0) {
+        s_misc[4] = 0;
+        s_misc[5] = -1;
       }
-      __syncthreads();
-      if (warp == 0) {  // threshold T: the k_eff-th smallest distance, and k_eff
-        constexpr int VPL = (BITS + 1 + 31) / 32;
-        int total = 0;
-#pragma unroll
-        for (int kk = 0; kk < VPL; ++kk) total += (lane + 32 * kk <= BITS) ? stv[lane + 32 * kk] : 0;
-#pragma unroll
-        for (int o2 = 16; o2 >= 1; o2 >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o2);
+      {
+        int x = 0;
+        if (tid <= BITS) {
+#pragma unroll 6
+          for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * (BITS + 1) + tid];
+        }
+        int total;
+        const int excl = block_excl_scan(x, s_scan, &total);
         const int k_eff = min(a.k, total);
-        int T = -1, run = 0;
-#pragma unroll
-        for (int kk = 0; kk < VPL; ++kk) {
-          const int v = lane + 32 * kk;
-          const int x = v <= BITS ? stv[v] : 0;
-          int incl = x;
-#pragma unroll
-          for (int o2 = 1; o2 < 32; o2 <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
-            if (lane >= o2) incl += y;
-          }
-          const int excl = run + incl - x;
-          const unsigned hit = __ballot_sync(0xFFFFFFFFu, x > 0 && excl < k_eff && excl + x >= k_eff);
-          if (hit && T < 0) {
-            const int src = __ffs(hit) - 1;
-            T = 32 * kk + src;
-            const int need = k_eff - __shfl_sync(0xFFFFFFFFu, excl, src);
-            if (lane == 0) s_misc[4] = need;
-          }
-          run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        if (x > 0 && excl < k_eff && excl + x >= k_eff) {   // exactly one thread
+          s_misc[5] = tid;
+          s_misc[4] = k_eff - excl;
         }
-        if (lane == 0) {
-          s_misc[5] = T;
-          s_misc[6] = k_eff;
-          if (T < 0) s_misc[4] = 0;
-        }
+        if (tid == 0) s_misc[6] = k_eff;
       }
       __syncthreads();
       {
@@ -1267,13 +1251,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       __syncthreads();
 
       if constexpr (MODE == kModeFused) {
-        for (int i = tid; i < RG * kD; i += NT) S.qf[i] *= a.scale_log2;
-        __syncthreads();
         attend_and_finish<RG>(a, unit, c, S.sel, my_sel, S.qf, S.scratch,
                               3u * static_cast<uint32_t>(a.C), s_misc);
       } else {
         if (tid == 0) {
-          __threadfence();
           const uint32_t old = atom_add_acq_rel(ctr, 1u);
           if (old == 3u * a.C - 1u) atomicExch(ctr, 0u);
         }
