@@ -530,9 +530,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
   S.scratch = smem + lay.scratch;
   int* s_scan = s_int;              // NWARPS + 1 entries
   int* s_misc = s_int + NWARPS + 1; // scalars
-  __shared__ __align__(8) unsigned long long s_rwbar;                       // R / W staging
+  __shared__ __align__(8) unsigned long long s_rwbar;                       // W staging
   const uint32_t rw_addr = smem_addr(&s_rwbar);
-  uint32_t rw_seq = 0;  // R/W phases used so far
+  uint32_t rw_seq = 0;  // W phases used so far
   if (tid == 0) {
     mbar_init(rw_addr, 1u);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -566,11 +566,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       continue;
     } else {
       // ---------------------------------------------------------- phase 0
-      // R reaches shared memory by one bulk copy on its mbarrier, requested
-      // before any metadata.  Every warp streams its own run of pages into a
-      // lane-private ring: the first kLaneSlots pages of each warp at once,
-      // the rest of the ring -- which shares its storage with R -- as soon
-      // as q~ = q R is formed.
+      // R reaches shared memory ahead of any metadata.  Every warp streams
+      // its own run of pages into a lane-private ring: the first kLaneSlots
+      // pages of each warp at once, the rest of the ring -- which shares its
+      // storage with R -- as soon as q~ = q R is formed.  W follows by bulk
+      // copy on an mbarrier once the ring has drained.
       const long long pb = static_cast<long long>(c) * a.NP / a.C;
       const long long pe = static_cast<long long>(c + 1) * a.NP / a.C;
       const int my_pages = static_cast<int>(pe - pb);
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
                      kD * sizeof(float), rw_addr);
         }
       };
-      // thread 0 waits for the next R/W phase; false (all threads) on timeout
+      // thread 0 waits for the next W phase; false (all threads) on timeout
       auto wait_rw = [&]() {
         const bool ok = (tid == 0) ? mbar_wait(rw_addr, rw_seq & 1u, a.spin_limit) : true;
         ++rw_seq;
@@ -631,23 +631,22 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         cp_async_commit();
       };
 
-      if (tid == 0) {
-        mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
-        bulk_g2s(smem_addr(sRW), Rg, kD * kD * sizeof(float), rw_addr);
-      }
+      {
+        // R alone first: 16-B pieces copied by every thread.  Requested
+        // together with the metadata it would land with the whole first
+        // burst; alone it lands in about one L2 round trip.
+        const uint4* src = reinterpret_cast<const uint4*>(Rg);
+        uint4* dst = reinterpret_cast<uint4*>(sRW);
 #pragma unroll
-      for (int gi = 0; gi < G0; ++gi) issue_group(gi);
+        for (int u = 0; u < kD * kD / 4 / NT; ++u) cp_async16(dst + tid + u * NT, src + tid + u * NT);
+        cp_async_commit();
+      }
       // queries of the group, as float (raw) -- q~ is derived from these
       for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
-      if (!wait_rw()) {
-        cp_async_wait<0>();
-        if (tid == 0) {
-          atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-          mbar_wait(rw_addr, (rw_seq - 1) & 1u, a.spin_limit);
-        }
-        __syncthreads();
-        return;
-      }
+      cp_async_wait<0>();    // this thread's pieces of R have landed
+      __syncthreads();       // ... and every thread's
+#pragma unroll
+      for (int gi = 0; gi < G0; ++gi) issue_group(gi);
       {
         float acc[RG];
         quarter_product<RG>(S.qf, sRW, acc);
