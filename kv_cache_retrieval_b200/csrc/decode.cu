@@ -45,8 +45,6 @@ namespace {
 constexpr int NT = kDecodeThreads;
 constexpr int NWARPS = NT / 32;
 
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
@@ -63,6 +61,11 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(d), "l"(gmem_src) : "memory");
+}
+// Copies 16 B when src_bytes is 16, writes 16 zero bytes when it is 0.
+__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(d), "l"(gmem_src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -104,15 +107,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
     if (mbar_try(bar, parity)) return true;
   } while (static_cast<unsigned long long>(clock64() - t0) <= limit);
   return false;
-}
-
-// Packed float32 pair multiply-add (one fma.rn.f32x2): d = a * b + c lane-wise.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
 }
 
 // Exclusive prefix sum over the CTA.  Every thread must call it.
@@ -240,6 +234,11 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
 }
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
 __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
                : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
@@ -281,147 +280,164 @@ struct Smem {
 
 // ----------------------------------------------------------------------------
 // Phase 6: attention of the r heads over `cnt` tokens listed in sel[], then
-// the per-unit merge.  sq: pre-scaled queries (scale * log2 e) [r][d].
+// the per-unit merge.
+//
+// Warp w takes tiles of 16 selected tokens (tiles w, w + 16, ...).  Their K
+// and V rows are staged in the warp's own 8 KB of shared memory (16-B chunk c
+// of token row r at position c ^ (r & 7), so that ldmatrix is conflict-free)
+// and both products run on the tensor cores with fp32 accumulation:
+//   S = Q K^T   m16n8k16, rows = the r heads (bf16 queries, unscaled, so
+//               the products are exact), columns = tokens;
+//   O += P V    rows 0-7 = the bf16 value of each head's softmax weights,
+//               rows 8-15 = the bf16 remainder, so P loses no precision.
+// Online softmax in float32 (exp2 with the scale folded in).  The next
+// tile's K is fetched during the softmax and P V, its V during the next Q K^T.
 template <int RG>
 __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const int* sel, int cnt,
-                                  const float* sq, unsigned char* scratch, uint32_t final_target,
-                                  int* s_int) {
+                                  unsigned char* scratch, uint32_t final_target, int* s_int) {
+  static_assert(RG <= 8, "the heads fill at most the upper 8 rows of an m16 tile");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int hf = lane >> 4, hl = lane & 15;
+  const int g8 = lane >> 2, t4 = lane & 3;      // mma fragment: row (head), column pair
+  const int lm = lane >> 3, lr = lane & 7;      // ldmatrix: matrix, row
+  const int b = unit / a.Hkv, g = unit % a.Hkv;
   const size_t unit_rows = static_cast<size_t>(unit) * a.n_cap;
   const uint16_t* Ku = a.K + unit_rows * kD;
   const uint16_t* Vu = a.V + unit_rows * kD;
 
-  // Half-warp hw attends tokens sel[hw], sel[hw + 32], ...  Its lane hl only
-  // uses the 16-B slices [8 hl, 8 hl + 8) of each K and V row, so it copies
-  // exactly those into its own slots (kAttnSlots tokens in flight) with
-  // cp.async and waits on its own copies: no barrier is involved.
-  const int hw_id = warp * 2 + hf;
-  uint4* kslot = reinterpret_cast<uint4*>(scratch) + hw_id * kAttnSlots * 16 + hl;
-  uint4* vslot = kslot + 32 * kAttnSlots * 16;
-  const int n_iter = cnt > warp * 2 ? (cnt - warp * 2 + 31) / 32 : 0;  // warp-uniform
-  const int n_pair = (n_iter + 1) / 2;
-  auto issue_pair = [&](int jp) {  // tokens 2 jp and 2 jp + 1 of this half-warp: one group
+  // Q fragments: row g8 = head g8 of the group (dims 16 ks + 2 t4, + 1 and
+  // 16 ks + 8 + 2 t4, + 1); rows 8-15 are zero
+  uint32_t qa[kD / 16][2];
+  {
+    const int hq = g8 < RG ? g8 : 0;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(a.q + (static_cast<size_t>(b) * a.Hq + g * RG + hq) * kD);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int j = 2 * jp + u;
-      const int t = hw_id + 32 * j;
-      if (j < n_iter && t < cnt) {
-        const size_t row = static_cast<size_t>(sel[t]) * kD + hl * 8;
-        cp_async16(kslot + (j % kAttnSlots) * 16, Ku + row);
-        cp_async16(vslot + (j % kAttnSlots) * 16, Vu + row);
+    for (int ks = 0; ks < kD / 16; ++ks) {
+      qa[ks][0] = g8 < RG ? __ldg(qrow + 8 * ks + t4) : 0u;
+      qa[ks][1] = g8 < RG ? __ldg(qrow + 8 * ks + 4 + t4) : 0u;
+    }
+  }
+
+  unsigned char* kbuf = scratch + warp * 8192;
+  unsigned char* vbuf = kbuf + 4096;
+  const uint32_t kb_s = smem_addr(kbuf), vb_s = smem_addr(vbuf);
+  const int n_tiles = (cnt + 15) / 16;
+  // every lane: 8 of the tile's 256 16-B chunks of K (or V), one commit group;
+  // rows past cnt are zero-filled
+  auto issue = [&](const uint16_t* base, unsigned char* buf, int tile) {
+    if (tile < n_tiles) {
+      const int ch = lane & 15;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = (lane >> 4) + 2 * i;
+        const int t = tile * 16 + r;
+        const bool ok = t < cnt;
+        const uint16_t* src = ok ? base + static_cast<size_t>(sel[t]) * kD + ch * 8 : base;
+        cp_async16_zfill(buf + r * 256 + ((ch ^ (r & 7)) << 4), src, ok ? 16u : 0u);
       }
     }
     cp_async_commit();
   };
 
-  float2 q[RG][4];
+  float o[kD / 8][4];
 #pragma unroll
-  for (int h = 0; h < RG; ++h)
+  for (int nt = 0; nt < kD / 8; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) q[h][e] = make_float2(sq[h * kD + hl * 8 + 2 * e], sq[h * kD + hl * 8 + 2 * e + 1]);
-  float m[RG], l[RG];
-  float2 o[RG][4];
-#pragma unroll
-  for (int h = 0; h < RG; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[h][e] = make_float2(0.f, 0.f);
-  }
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
 
+  issue(Ku, kbuf, warp);
+  issue(Vu, vbuf, warp);
+  for (int tile = warp; tile < n_tiles; tile += NWARPS) {
+    cp_async_wait<1>();   // this lane's K chunks of the tile
+    __syncwarp();         // ... and every lane's
+    float sacc[2][4];
 #pragma unroll
-  for (int jp = 0; jp < kAttnSlots / 2; ++jp) issue_pair(jp);
-  for (int jp = 0; jp < n_pair; ++jp) {
-    cp_async_wait<kAttnSlots / 2 - 1>();   // this lane's slices of the pair have landed
-    const int j0 = 2 * jp;
-    const bool va = hw_id + 32 * j0 < cnt;          // uniform within a half-warp
-    const bool vb = hw_id + 32 * (j0 + 1) < cnt;
-    uint4 ka = make_uint4(0u, 0u, 0u, 0u), kb = ka, xa = ka, xb = ka;
-    if (va) {
-      ka = kslot[(j0 % kAttnSlots) * 16];
-      xa = vslot[(j0 % kAttnSlots) * 16];
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(kb_s + ((lm >> 1) * 8 + lr) * 256 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4),
+              b0, b1, b2, b3);
+      mma_bf16_16816(sacc[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+      mma_bf16_16816(sacc[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
     }
-    if (vb) {
-      kb = kslot[((j0 + 1) % kAttnSlots) * 16];
-      xb = vslot[((j0 + 1) % kAttnSlots) * 16];
-    }
-    issue_pair(jp + kAttnSlots / 2);   // refill the slots just read
-    const uint32_t kwa[4] = {ka.x, ka.y, ka.z, ka.w}, kwb[4] = {kb.x, kb.y, kb.z, kb.w};
-    const uint32_t vwa[4] = {xa.x, xa.y, xa.z, xa.w}, vwb[4] = {xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-    for (int h = 0; h < RG; ++h) {
-      float2 da = make_float2(0.f, 0.f), db = da;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        da = ffma2(q[h][e], make_float2(bf_lo(kwa[e]), bf_hi(kwa[e])), da);
-        db = ffma2(q[h][e], make_float2(bf_lo(kwb[e]), bf_hi(kwb[e])), db);
-      }
-      float sa = da.x + da.y, sb = db.x + db.y;
-      // butterflies over the 16 lanes of this half-warp: every lane ends
-      // with the same (commutative) sums
-#pragma unroll
-      for (int o2 = 8; o2 >= 1; o2 >>= 1) {
-        sa += __shfl_xor_sync(0xFFFFFFFFu, sa, o2);
-        sb += __shfl_xor_sync(0xFFFFFFFFu, sb, o2);
-      }
-      const float mn = fmaxf(m[h], fmaxf(va ? sa : -INFINITY, vb ? sb : -INFINITY));
-      if (mn != -INFINITY) {
-        const float alpha = exp2f(m[h] - mn);      // 0 when m was -inf
-        const float pa = va ? exp2f(sa - mn) : 0.f;
-        const float pb = vb ? exp2f(sb - mn) : 0.f;
-        l[h] = fmaf(l[h], alpha, pa + pb);
-        const float2 al = make_float2(alpha, alpha), p2a = make_float2(pa, pa), p2b = make_float2(pb, pb);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float2 t2 = make_float2(o[h][e].x * al.x, o[h][e].y * al.y);
-          t2 = ffma2(p2a, make_float2(bf_lo(vwa[e]), bf_hi(vwa[e])), t2);
-          o[h][e] = ffma2(p2b, make_float2(bf_lo(vwb[e]), bf_hi(vwb[e])), t2);
-        }
-        m[h] = mn;
-      }
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();
+    __syncwarp();
+    issue(Ku, kbuf, tile + NWARPS);
 
-  // fold the two half-warps of each warp together, then merge the 16 warp
-  // states through shared memory: [warp][h][d + 2]
-#pragma unroll
-  for (int h = 0; h < RG; ++h) {
-    const float mo = __shfl_xor_sync(0xFFFFFFFFu, m[h], 16);
-    const float lo = __shfl_xor_sync(0xFFFFFFFFu, l[h], 16);
-    const float M = fmaxf(m[h], mo);
-    const float wa = (M == -INFINITY) ? 0.f : exp2f(m[h] - M);
-    const float wb = (M == -INFINITY) ? 0.f : exp2f(mo - M);
-    l[h] = l[h] * wa + lo * wb;
+    // head g8's scores of tokens 2 t4, 2 t4 + 1, 8 + 2 t4, 9 + 2 t4
+    const int valid = cnt - tile * 16;
+    float sc[4] = {sacc[0][0], sacc[0][1], sacc[1][0], sacc[1][1]};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float ox = __shfl_xor_sync(0xFFFFFFFFu, o[h][e].x, 16);
-      const float oy = __shfl_xor_sync(0xFFFFFFFFu, o[h][e].y, 16);
-      o[h][e] = make_float2(o[h][e].x * wa + ox * wb, o[h][e].y * wa + oy * wb);
+      const int tok = (e >> 1) * 8 + 2 * t4 + (e & 1);
+      sc[e] = tok < valid ? sc[e] * a.scale_log2 : -INFINITY;
     }
-    m[h] = M;
-  }
-  float* mer = reinterpret_cast<float*>(scratch);
-  if (hf == 0) {
+    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);       // finite: the tile has a valid token
+    const float alpha = exp2f(m_run - m_new);   // 0 while m_run is -inf
+    float pr[4];
 #pragma unroll
-    for (int h = 0; h < RG; ++h) {
-      float* dst = mer + (warp * RG + h) * (kD + 2);
+    for (int e = 0; e < 4; ++e) pr[e] = exp2f(sc[e] - m_new);
+    float ps = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
+    l_run = fmaf(l_run, alpha, ps);
+    m_run = m_new;
+    uint32_t pa[4];
+    {
+      uint16_t hi[4], lo[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        dst[hl * 8 + 2 * e] = o[h][e].x;
-        dst[hl * 8 + 2 * e + 1] = o[h][e].y;
+        const __nv_bfloat16 h16 = __float2bfloat16_rn(pr[e]);
+        hi[e] = __bfloat16_as_ushort(h16);
+        lo[e] = __bfloat16_as_ushort(__float2bfloat16_rn(pr[e] - __bfloat162float(h16)));
       }
-      if (hl == 0) {
-        dst[kD] = m[h];
-        dst[kD + 1] = l[h];
-      }
+      pa[0] = hi[0] | (static_cast<uint32_t>(hi[1]) << 16);   // row g8, tokens 2 t4, + 1
+      pa[1] = lo[0] | (static_cast<uint32_t>(lo[1]) << 16);   // row g8 + 8
+      pa[2] = hi[2] | (static_cast<uint32_t>(hi[3]) << 16);   // row g8, tokens 8 + 2 t4, + 1
+      pa[3] = lo[2] | (static_cast<uint32_t>(lo[3]) << 16);
+    }
+#pragma unroll
+    for (int nt = 0; nt < kD / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][e] *= alpha;
+
+    cp_async_wait<1>();   // this lane's V chunks of the tile
+    __syncwarp();
+#pragma unroll
+    for (int np = 0; np < kD / 16; ++np) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(vb_s + ((lm & 1) * 8 + lr) * 256 + (static_cast<uint32_t>((2 * np + (lm >> 1)) ^ lr) << 4),
+                    b0, b1, b2, b3);
+      mma_bf16_16816(o[2 * np], pa[0], pa[1], pa[2], pa[3], b0, b1);
+      mma_bf16_16816(o[2 * np + 1], pa[0], pa[1], pa[2], pa[3], b2, b3);
+    }
+    __syncwarp();
+    issue(Vu, vbuf, tile + NWARPS);
+  }
+  cp_async_wait<0>();
+  __syncthreads();   // the merge buffer below overlays the K / V tiles
+
+  // merge the 16 warp states through shared memory: [warp][h][d + 2]
+  float* mer = reinterpret_cast<float*>(scratch);
+  if (g8 < RG) {
+    float* dst = mer + (warp * RG + g8) * (kD + 2);
+#pragma unroll
+    for (int nt = 0; nt < kD / 8; ++nt) {
+      dst[8 * nt + 2 * t4] = o[nt][0] + o[nt][2];
+      dst[8 * nt + 2 * t4 + 1] = o[nt][1] + o[nt][3];
+    }
+    if (t4 == 0) {
+      dst[kD] = m_run;
+      dst[kD + 1] = l_run;
     }
   }
   __syncthreads();
 
-  const int b = unit / a.Hkv, g = unit % a.Hkv;
   constexpr int PS = part_stride(RG);
   float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * PS;
   // weights e^(m_w - M) of the 16 warp states and the CTA max / sum, per head
@@ -550,18 +566,14 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
     const uint16_t* qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * RG) * kD;
 
     if constexpr (MODE == kModeAttend) {
-      for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
-      __syncthreads();
       const int n = a.nsel_in[unit];
       const int s0 = static_cast<int>(static_cast<long long>(c) * n / a.C);
       const int s1 = static_cast<int>(static_cast<long long>(c + 1) * n / a.C);
       const int32_t* src = a.tok_in + static_cast<size_t>(unit) * a.k;
 #pragma unroll 8
       for (int i = s0 + tid; i < s1; i += NT) S.sel[i - s0] = src[i];
-      for (int i = tid; i < RG * kD; i += NT) S.qf[i] *= a.scale_log2;
       __syncthreads();
-      attend_and_finish<RG>(a, unit, c, S.sel, s1 - s0, S.qf, S.scratch,
-                            static_cast<uint32_t>(a.C), s_misc);
+      attend_and_finish<RG>(a, unit, c, S.sel, s1 - s0, S.scratch, static_cast<uint32_t>(a.C), s_misc);
       __syncthreads();
       continue;
     } else {
@@ -810,11 +822,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         }
         __syncthreads();
         return;
-      }
-      if constexpr (MODE == kModeFused) {
-        // the raw queries have served q~ and the codes: pre-scale them for
-        // attention while the unit barrier completes
-        for (int i = tid; i < RG * kD; i += NT) S.qf[i] *= a.scale_log2;
       }
       if (tid == 0) {
         int ok = 1;
@@ -1250,8 +1257,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       __syncthreads();
 
       if constexpr (MODE == kModeFused) {
-        attend_and_finish<RG>(a, unit, c, S.sel, my_sel, S.qf, S.scratch,
-                              3u * static_cast<uint32_t>(a.C), s_misc);
+        attend_and_finish<RG>(a, unit, c, S.sel, my_sel, S.scratch, 3u * static_cast<uint32_t>(a.C), s_misc);
       } else {
         if (tid == 0) {
           const uint32_t old = atom_add_acq_rel(ctr, 1u);

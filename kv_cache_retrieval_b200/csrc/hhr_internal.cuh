@@ -18,7 +18,6 @@ constexpr int kBuckets = 2048;          // page top-P histogram bins
 constexpr int kCandMax = 1024;          // boundary-bucket candidates held in shared memory
 constexpr int kRankDirect = 48;         // at most this many are ranked without a second level
 constexpr int kMaxTokensPerCta = 16384; // candidate tokens one CTA scores
-constexpr int kAttnSlots = 8;           // K/V tokens in flight per half-warp
 constexpr int kLaneSlots = 16;         // ring slots per warp below the R / W buffer (8 KiB)
 constexpr int kRingSlots = 24;         // ring slots per warp in all (12 KiB), the upper 8 over R / W
 constexpr unsigned long long kSpinLimit = 1ull << 31;  // ~1 s at 2 GHz
@@ -112,7 +111,7 @@ inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, 
     hist = sizeof(int) * ((size_t)C * (bits + 1) + 2 * (size_t)C) + 16;
   }
   if (mode != kModeSelect) {
-    const size_t ring = (size_t)32 * kAttnSlots * 16 * 2 * 16;  // half-warps x slots x lanes x (K, V) x 16 B
+    const size_t ring = (size_t)(kDecodeThreads / 32) * 2 * 16 * 2 * kD;  // per warp: K and V of 16 tokens
     size_t merge = sizeof(float) * ((kDecodeThreads / 32) * (size_t)r * (kD + 2) + (kDecodeThreads / 32) * (size_t)r + 2 * (size_t)r);
     const size_t parts = sizeof(float) * ((size_t)C * part_stride(r) + (size_t)C * r + r);  // final merge
     merge = merge > parts ? merge : parts;
