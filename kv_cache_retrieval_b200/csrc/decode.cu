@@ -440,31 +440,21 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
 
   constexpr int PS = part_stride(RG);
   float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * PS;
-  // weights e^(m_w - M) of the 16 warp states and the CTA max / sum, per head
-  float* mw = mer + NWARPS * RG * (kD + 2);   // [NWARPS][RG] weights, then [RG] M, [RG] L
-  if (warp < RG) {
-    const int h = warp;
-    const float mv = lane < NWARPS ? mer[(lane * RG + h) * (kD + 2) + kD] : -INFINITY;
-    float M = mv;
-#pragma unroll
-    for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
-    const float wgt = (lane < NWARPS && M != -INFINITY) ? exp2f(mv - M) : 0.f;
-    float L = lane < NWARPS ? mer[(lane * RG + h) * (kD + 2) + kD + 1] * wgt : 0.f;
-#pragma unroll
-    for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
-    if (lane < NWARPS) mw[lane * RG + h] = wgt;
-    if (lane == 0) {
-      mw[NWARPS * RG + h] = M;
-      mw[NWARPS * RG + RG + h] = L;
-    }
-  }
-  __syncthreads();
+  // thread (h, j): the 16 warp states of head h combined with weights
+  // e^(m_w - M), M the largest m_w (every thread of the head derives them)
   for (int oi = tid; oi < RG * kD; oi += NT) {
     const int h = oi / kD, j = oi % kD;
-    float O = 0.f;
+    float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NWARPS; ++w) O = fmaf(mer[(w * RG + h) * (kD + 2) + j], mw[w * RG + h], O);
-    const float M = mw[NWARPS * RG + h], L = mw[NWARPS * RG + RG + h];
+    for (int w = 0; w < NWARPS; ++w) M = fmaxf(M, mer[(w * RG + h) * (kD + 2) + kD]);
+    float O = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w) {
+      const float* src = mer + (w * RG + h) * (kD + 2);
+      const float wgt = (M == -INFINITY) ? 0.f : exp2f(src[kD] - M);
+      O = fmaf(src[j], wgt, O);
+      L = fmaf(src[kD + 1], wgt, L);
+    }
     if (a.C == 1) {
       a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
     } else {
@@ -493,33 +483,21 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     for (int i = tid; i < n4; i += NT)
       reinterpret_cast<float4*>(sp)[i] = __ldcg(reinterpret_cast<const float4*>(parts) + i);
     __syncthreads();
-    // weights e^(m_c - M) of every CTA's state and 1 / sum, once per head
-    float* sw = sp + a.C * PS;              // [C][RG]
-    float* sinv = sw + a.C * RG;            // [RG]
-    if (warp < RG) {
-      const int h = warp;
-      float M = -INFINITY;
-      for (int cc = lane; cc < a.C; cc += 32) M = fmaxf(M, sp[cc * PS + h * (kD + 2) + kD]);
-#pragma unroll
-      for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
-      float L = 0.f;
-      for (int cc = lane; cc < a.C; cc += 32) {
-        const float* src = sp + cc * PS + h * (kD + 2);
-        const float wgt = (M == -INFINITY) ? 0.f : exp2f(src[kD] - M);
-        sw[cc * RG + h] = wgt;
-        L = fmaf(src[kD + 1], wgt, L);
-      }
-#pragma unroll
-      for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
-      if (lane == 0) sinv[h] = (L > 0.f) ? 1.f / L : 0.f;
-    }
-    __syncthreads();
+    // thread (h, j): the C states of head h combined the same way
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
-      float O = 0.f;
+      float M = -INFINITY;
 #pragma unroll 6
-      for (int cc = 0; cc < a.C; ++cc) O = fmaf(sp[cc * PS + h * (kD + 2) + j], sw[cc * RG + h], O);
-      a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = O * sinv[h];
+      for (int cc = 0; cc < a.C; ++cc) M = fmaxf(M, sp[cc * PS + h * (kD + 2) + kD]);
+      float O = 0.f, L = 0.f;
+#pragma unroll 6
+      for (int cc = 0; cc < a.C; ++cc) {
+        const float* src = sp + cc * PS + h * (kD + 2);
+        const float wgt = (M == -INFINITY) ? 0.f : exp2f(src[kD] - M);
+        O = fmaf(src[j], wgt, O);
+        L = fmaf(src[kD + 1], wgt, L);
+      }
+      a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
     }
   }
   if (tid == 0) atomicExch(a.counters + unit, 0u);
