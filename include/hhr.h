@@ -119,12 +119,25 @@ const char* hhr_status_string(int32_t status);
  *         the same bytes as encoding the page in one call.  A page starting at
  *         or after n_begin is overwritten.
  * Requires 0 <= n_begin <= n_end <= n_cap; n_begin == n_end enqueues nothing.
- * Keys are encoded to float32 accuracy: each rotated and projected value is a
- * float32 dot product of the bf16 key with the f32 column.
+ * Keys are encoded to float32 accuracy: the products run on the tensor cores
+ * with each f32 weight entered as three bf16 terms whose sum is exactly the
+ * weight (so every product with a bf16 key is exact) and f32 accumulation.
+ * The kernel's internal pipeline waits are bounded (about one second); one
+ * that runs out abandons the call and sets a sticky HHR_ERR_TIMEOUT, read
+ * with hhr_encode_status().
  */
 int32_t hhr_encode_keys(const hhr_dims* dims, const void* K, const float* R, const float* W,
                         int32_t n_begin, int32_t n_end, uint32_t* codes, void* meta,
                         void* stream);
+
+/*
+ * Waits for `stream`, returns the sticky status of the key-encoding kernels
+ * on the current device (HHR_OK, or HHR_ERR_TIMEOUT after an abandoned
+ * hhr_encode_keys) and clears it.  Returns HHR_ERR_CUDA if the copy or the
+ * wait fails.  No counterpart in the paper: it reports the kernel's bounded
+ * waits.
+ */
+int32_t hhr_encode_status(void* stream);
 
 /*
  * Bytes of device workspace hhr_select / hhr_sparse_attend / hhr_decode_step

@@ -60,6 +60,7 @@ _SIGS = {
     "hhr_decode_step_noalloc": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
                                        _I32, C.c_float, _P, _P, _P, _P, _P]),
     "hhr_read_status": (_I32, [_P, _P]),
+    "hhr_encode_status": (_I32, [_P]),
     "hhr_test_wait_timeout": (_I32, [_P, C.c_size_t, C.c_uint64, _P]),
 }
 
@@ -171,6 +172,14 @@ def hhr_read_status(workspace, stream=None) -> int:
     st = lib().hhr_read_status(_ptr(workspace), _stream(stream))
     if st == HHR_ERR_CUDA:
         raise HhrError(st, "hhr_read_status")
+    return st
+
+
+def hhr_encode_status(stream=None) -> int:
+    """Sticky status of the key-encoding kernels (HHR_OK or HHR_ERR_TIMEOUT), cleared after reading."""
+    st = lib().hhr_encode_status(_stream(stream))
+    if st == HHR_ERR_CUDA:
+        raise HhrError(st, "hhr_encode_status")
     return st
 
 

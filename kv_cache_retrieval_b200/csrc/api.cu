@@ -180,10 +180,13 @@ int32_t hhr_encode_keys(const hhr_dims* dims, const void* K, const float* R, con
   a.np_cap = np_cap_of(dims);
   a.n_begin = n_begin;
   a.n_end = n_end;
-  a.tile_begin = n_begin / 64 * 64;
-  a.n_tiles = (n_end - a.tile_begin + 63) / 64;
-  if (a.units > 65535) return HHR_ERR_UNSUPPORTED;
-  return finish_launch(launch_encode(a, static_cast<cudaStream_t>(stream)));
+  a.tile_begin = n_begin / kEncodeTileKeys * kEncodeTileKeys;
+  a.n_tiles = (n_end - a.tile_begin + kEncodeTileKeys - 1) / kEncodeTileKeys;
+  DeviceInfo info;
+  if (int32_t st = device_info(&info)) return st;
+  if (encode_smem_bytes() > info.smem_optin) return HHR_ERR_UNSUPPORTED;
+  if (static_cast<long long>(a.units / a.Hkv) * a.n_tiles > 0x7FFFFFFFLL) return HHR_ERR_UNSUPPORTED;
+  return finish_launch(launch_encode(a, info.sms, static_cast<cudaStream_t>(stream)));
 }
 
 size_t hhr_workspace_size(const hhr_dims* dims, int32_t P, int32_t k) {
@@ -264,6 +267,12 @@ int32_t hhr_decode_step(const hhr_dims* dims, const void* q, const float* R, con
   return decode_common(dims, kModeFused, q, R, W, codes, meta, K, V, nullptr, nullptr, n_valid, P,
                        k, scale, page_idx, tok_idx, n_sel, out, nullptr, nullptr, workspace,
                        ws_bytes, stream);
+}
+
+int32_t hhr_encode_status(void* stream) {
+  uint32_t host = 0;
+  if (encode_read_status(&host, static_cast<cudaStream_t>(stream)) != cudaSuccess) return HHR_ERR_CUDA;
+  return static_cast<int32_t>(host);
 }
 
 int32_t hhr_read_status(void* workspace, void* stream) {

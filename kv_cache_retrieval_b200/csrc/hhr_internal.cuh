@@ -140,7 +140,11 @@ inline __host__ __device__ DecodeSmem decode_smem(int NP, int C, int bits, int r
 // Launchers (defined in decode.cu / encode.cu).  Return a cudaError_t.
 cudaError_t launch_decode(const DecodeArgs& a, int r, int bits, int mode, size_t smem_bytes,
                           cudaStream_t stream);
-cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t stream);
+cudaError_t launch_encode(const EncodeArgs& a, int sms, cudaStream_t stream);
+size_t encode_smem_bytes();
+// Copies the encode kernels' sticky error word to *out and clears it (synchronizes `stream`).
+cudaError_t encode_read_status(uint32_t* out, cudaStream_t stream);
+constexpr int kEncodeTileKeys = 128;   // keys per encode tile (tile starts are multiples of it)
 cudaError_t launch_wait_timeout(uint32_t* status, uint32_t* counter, unsigned long long spin,
                                 cudaStream_t stream);
 
