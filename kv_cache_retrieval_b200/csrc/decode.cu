@@ -202,6 +202,27 @@ __device__ void find_boundary(const int* hist, int need, int* s_warp, int* out) 
   __syncthreads();
 }
 
+// Thread 0 waits until the unit counter reaches `target` (acquire), then the
+// CTA barrier releases everyone.  Returns false (HHR_ERR_TIMEOUT recorded)
+// if the wait ran out.  Every thread of the CTA calls it.
+__device__ bool unit_wait(const uint32_t* ctr, uint32_t target, const DecodeArgs& a, int* s_flag) {
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const long long t0 = clock64();
+    while (ld_acquire(ctr) < target) {
+      if (static_cast<unsigned long long>(clock64() - t0) > a.spin_limit) {
+        atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+    *s_flag = ok;
+  }
+  __syncthreads();
+  return *s_flag != 0;
+}
+
 // One quarter of x[r][d] . M[d][d] (both float32 in shared memory): thread t
 // returns, for every head h, the sum over rows i in [32 (t / 128), 32 (t / 128) + 32)
 // of x[h][i] * M[i][t % 128].  M is read once per CTA, conflict-free; x by
@@ -539,6 +560,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
 
   for (int unit = blockIdx.x / a.C; unit < a.units; unit += a.grid_units) {
     const int b = unit / a.Hkv, g = unit % a.Hkv;
+
     uint32_t* ctr = a.counters + unit;
 
     const uint16_t* qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * RG) * kD;
@@ -801,21 +823,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         __syncthreads();
         return;
       }
-      if (tid == 0) {
-        int ok = 1;
-        const long long t0 = clock64();
-        while (ld_acquire(ctr) < static_cast<uint32_t>(a.C)) {
-          if (static_cast<unsigned long long>(clock64() - t0) > a.spin_limit) {
-            atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-            ok = 0;
-            break;
-          }
-          __nanosleep(32);
-        }
-        s_misc[0] = ok;
-      }
-      __syncthreads();
-      if (!s_misc[0]) return;
+      if (!unit_wait(ctr, static_cast<uint32_t>(a.C), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 2
       const int NP = a.NP, Pk = a.Pk;
@@ -877,9 +885,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         const float gmin = s_flt[0];
         const float range = s_flt[1] - gmin;
         const float inv = (range > 0.f && range <= FLT_MAX) ? static_cast<float>(kBuckets) / range : 0.f;
+        // bin = round((u - gmin) * inv) by one FMA: the 1.5 * 2^23 offset
+        // leaves the rounded integer in the low mantissa bits.  Monotone in u,
+        // and histogram and extraction use the same map, which is all the
+        // selection needs; clamped for any input (NaN included).
         auto bucket = [&](float u) {
-          const int bk = static_cast<int>((u - gmin) * inv);
-          return bk < kBuckets - 1 ? bk : kBuckets - 1;
+          const int bk = __float_as_int(fmaf(u - gmin, inv, 12582912.f)) - 0x4B400000;
+          return min(max(bk, 0), kBuckets - 1);
         };
 #pragma unroll
         for (int u = 0; u < kU4; ++u) {
@@ -967,8 +979,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
             const float r2 = cmax - cmin;
             const float inv2 = (r2 > 0.f && r2 <= FLT_MAX) ? static_cast<float>(kBuckets) / r2 : 0.f;
             auto bucket2 = [&](float u) {
-              const int bk = static_cast<int>((u - cmin) * inv2);
-              return bk < kBuckets - 1 ? bk : kBuckets - 1;
+              const int bk = __float_as_int(fmaf(u - cmin, inv2, 12582912.f)) - 0x4B400000;
+              return min(max(bk, 0), kBuckets - 1);
             };
             for (int i = tid; i < nc; i += NT) atomicAdd(&sHist[bucket2(sCU[i])], 1);
             __syncthreads();
@@ -1096,21 +1108,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       // row through the CTA barrier)
       __syncthreads();
       if (tid == 0) atom_add_acq_rel(ctr, 1u);
-      if (tid == 0) {
-        int ok = 1;
-        const long long t0 = clock64();
-        while (ld_acquire(ctr) < 2u * static_cast<uint32_t>(a.C)) {
-          if (static_cast<unsigned long long>(clock64() - t0) > a.spin_limit) {
-            atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-            ok = 0;
-            break;
-          }
-          __nanosleep(32);
-        }
-        s_misc[0] = ok;
-      }
-      __syncthreads();
-      if (!s_misc[0]) return;
+      if (!unit_wait(ctr, 2u * static_cast<uint32_t>(a.C), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 5
       int* sHA = reinterpret_cast<int*>(S.scratch);  // [C][BITS + 1]
