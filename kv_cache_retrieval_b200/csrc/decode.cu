@@ -91,6 +91,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Brings the 128-B line holding `p` into L2 (no register result).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+}
+
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
@@ -1021,6 +1026,20 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         }
       }
       __syncthreads();
+      {
+        // the codes of the kept pages of this CTA's own page range into L2:
+        // the compaction below hands them to some CTA's Hamming pass, whose
+        // loads then hit L2 (a hint only; rows clamped to the codes buffer)
+        const size_t row_bytes = static_cast<size_t>(WORDS) * 4;
+        const char* cbase = reinterpret_cast<const char*>(a.codes + static_cast<size_t>(unit) * a.n_cap * WORDS);
+        for (long long p = pb + tid; p < pe; p += NT) {
+          if ((sBits[p >> 5] >> (p & 31)) & 1u) {
+            const size_t b0 = static_cast<size_t>(p) * a.page * row_bytes;
+            const size_t b1 = min(static_cast<size_t>(p + 1) * a.page, static_cast<size_t>(a.n_cap)) * row_bytes;
+            for (size_t off = b0 & ~static_cast<size_t>(127); off < b1; off += 128) prefetch_l2(cbase + off);
+          }
+        }
+      }
 
       // ---------------------------------------------------------- phase 3
       const int ks = static_cast<int>(static_cast<long long>(c) * Pk / a.C);
