@@ -648,20 +648,23 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
         cp_async_commit();
       };
 
-      {
-        // R alone first: 16-B pieces copied by every thread.  Requested
-        // together with the metadata it would land with the whole first
-        // burst; alone it lands in about one L2 round trip.
-        const uint4* src = reinterpret_cast<const uint4*>(Rg);
-        uint4* dst = reinterpret_cast<uint4*>(sRW);
-#pragma unroll
-        for (int u = 0; u < kD * kD / 4 / NT; ++u) cp_async16(dst + tid + u * NT, src + tid + u * NT);
-        cp_async_commit();
+      // R alone first, one bulk copy: requested together with the metadata
+      // it would land only with the whole first burst
+      if (tid == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
+        bulk_g2s(smem_addr(sRW), Rg, kD * kD * sizeof(float), rw_addr);
       }
       // queries of the group, as float (raw) -- q~ is derived from these
       for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
-      cp_async_wait<0>();    // this thread's pieces of R have landed
-      __syncthreads();       // ... and every thread's
+      if (!wait_rw()) {
+        if (tid == 0) {
+          atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+          mbar_wait(rw_addr, (rw_seq - 1) & 1u, a.spin_limit);   // the copy may still be in flight
+        }
+        __syncthreads();
+        return;
+      }
 #pragma unroll
       for (int gi = 0; gi < G0; ++gi) issue_group(gi);
       {
