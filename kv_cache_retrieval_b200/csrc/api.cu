@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "hhr.h"
 #include "hhr_internal.cuh"
@@ -43,15 +44,32 @@ struct DeviceInfo {
   size_t smem_optin = 0;
 };
 
+// SM count and opt-in shared memory of the current device, queried once per
+// device.
 int32_t device_info(DeviceInfo* info) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HHR_ERR_CUDA;
+  static std::mutex mu;
+  static DeviceInfo cache[kMaxDevices];
+  static bool known[kMaxDevices];
+  if (dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (known[dev]) {
+      *info = cache[dev];
+      return HHR_OK;
+    }
+  }
   int v = 0;
   if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return HHR_ERR_CUDA;
   info->sms = v;
   if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return HHR_ERR_CUDA;
   info->smem_optin = static_cast<size_t>(v);
+  if (dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(mu);
+    cache[dev] = *info;
+    known[dev] = true;
+  }
   return HHR_OK;
 }
 

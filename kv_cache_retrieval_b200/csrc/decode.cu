@@ -623,9 +623,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
       const long long wpe = pb + static_cast<long long>(my_pages) * (warp + 1) / NWARPS;
       const int w_pages = static_cast<int>(wpe - wpb);
       constexpr int PPG = 8;                        // pages per ring group; an A tile is two groups
-      constexpr int G0 = kLaneSlots / PPG;          // groups in flight while q~ is formed
+      constexpr int G0 = 1;                         // groups in flight while q~ is formed (A/B: 1 beats 0 and 2)
       constexpr int GR = kRingSlots / PPG;          // groups in flight afterwards
-      static_assert(kLaneSlots % PPG == 0 && kRingSlots % PPG == 0, "whole groups per ring");
+      static_assert(kLaneSlots % PPG == 0 && kRingSlots % PPG == 0 && G0 * PPG <= kLaneSlots,
+                    "whole groups per ring; the groups issued before q~ stay below the R / W buffer");
       static_assert(GR == 3, "tile ti reads groups 2 ti, 2 ti + 1 and refills them with 2 ti + 3, 2 ti + 4");
       static_assert((kRingSlots - kLaneSlots) * NWARPS * 512 == kD * kD * sizeof(float),
                     "the upper ring slots fill the R / W buffer exactly");
@@ -1282,8 +1283,8 @@ __global__ void wait_timeout_kernel(uint32_t* status, uint32_t* counter, unsigne
 template <int RG, int WORDS, int MODE>
 cudaError_t launch_t(const DecodeArgs& a, size_t smem, cudaStream_t stream) {
   auto kern = decode_kernel<RG, WORDS, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static std::atomic<size_t> raised[kMaxDevices];
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem, raised);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.grid_units * a.C));

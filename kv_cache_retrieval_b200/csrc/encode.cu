@@ -397,8 +397,8 @@ size_t encode_smem_bytes() { return static_cast<size_t>(kTerms + kStages) * kOpB
 
 cudaError_t launch_encode(const EncodeArgs& a, int sms, cudaStream_t stream) {
   const size_t smem = encode_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static std::atomic<size_t> raised[kMaxDevices];
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(encode_kernel), smem, raised);
   if (e != cudaSuccess) return e;
   const int n_ob = 1 + a.bits / kD;
   const int groups = a.Hkv * n_ob;

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstddef>
+#include <atomic>
 #include <cstdint>
 
 #include <cuda_runtime.h>
@@ -135,6 +136,25 @@ inline __host__ __device__ DecodeSmem decode_smem(int NP, int C, int bits, int r
   s.scratch = off;  off += align_up(decode_scratch_bytes(NP, C, bits, r, mode), 16);
   s.total = off;
   return s;
+}
+
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device, calling cudaFuncSetAttribute only when the limit grows
+// (one record per kernel and device: `raised` must be a zero-initialised
+// static array of kMaxDevices entries).
+constexpr int kMaxDevices = 64;
+inline cudaError_t ensure_smem_limit(const void* kernel, size_t bytes, std::atomic<size_t>* raised) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < kMaxDevices && raised[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess && dev < kMaxDevices) {
+    size_t cur = raised[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !raised[dev].compare_exchange_weak(cur, bytes, std::memory_order_release)) {
+    }
+  }
+  return e;
 }
 
 // Launchers (defined in decode.cu / encode.cu).  Return a cudaError_t.
