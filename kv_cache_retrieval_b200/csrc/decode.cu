@@ -304,6 +304,30 @@ struct Smem {
   unsigned char* scratch;
 };
 
+// One warp: the merge weights of n partial softmax states of one head.
+// State i has its running max at st[i * stride + d] and its sum at
+// st[i * stride + d + 1].  Writes wgt[i] = 2^(m_i - M) (M the largest m_i;
+// zero when every state is empty) and hdr = {M, sum_i wgt[i] l_i}.
+__device__ __forceinline__ void merge_weights(const float* st, int stride, int n, float* wgt, float* hdr) {
+  const int lane = threadIdx.x & 31;
+  float M = -INFINITY;
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, st[i * stride + kD]);
+#pragma unroll
+  for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
+  float L = 0.f;
+  for (int i = lane; i < n; i += 32) {
+    const float w = (M == -INFINITY) ? 0.f : exp2f(st[i * stride + kD] - M);
+    wgt[i] = w;
+    L = fmaf(st[i * stride + kD + 1], w, L);
+  }
+#pragma unroll
+  for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
+  if (lane == 0) {
+    hdr[0] = M;
+    hdr[1] = L;
+  }
+}
+
 // ----------------------------------------------------------------------------
 // Phase 6: attention of the r heads over `cnt` tokens listed in sel[], then
 // the per-unit merge.
@@ -329,19 +353,6 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   const size_t unit_rows = static_cast<size_t>(unit) * a.n_cap;
   const uint16_t* Ku = a.K + unit_rows * kD;
   const uint16_t* Vu = a.V + unit_rows * kD;
-
-  // Q fragments: row g8 = head g8 of the group (dims 16 ks + 2 t4, + 1 and
-  // 16 ks + 8 + 2 t4, + 1); rows 8-15 are zero
-  uint32_t qa[kD / 16][2];
-  {
-    const int hq = g8 < RG ? g8 : 0;
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(a.q + (static_cast<size_t>(b) * a.Hq + g * RG + hq) * kD);
-#pragma unroll
-    for (int ks = 0; ks < kD / 16; ++ks) {
-      qa[ks][0] = g8 < RG ? __ldg(qrow + 8 * ks + t4) : 0u;
-      qa[ks][1] = g8 < RG ? __ldg(qrow + 8 * ks + 4 + t4) : 0u;
-    }
-  }
 
   unsigned char* kbuf = scratch + warp * 8192;
   unsigned char* vbuf = kbuf + 4096;
@@ -373,6 +384,19 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
 
   issue(Ku, kbuf, warp);
   issue(Vu, vbuf, warp);
+  // The group's queries as the A tile of Q K^T in shared memory (above the
+  // warps' K / V buffers): row h < r is head h, rows r..15 are zero; 16-B
+  // chunk c of row h sits at c ^ (h & 7).  Fragments are read per k-step
+  // with ldmatrix rather than held in registers.
+  unsigned char* qtile = scratch + NWARPS * 8192;
+  if (tid < 16 * 16) {
+    const int h = tid >> 4, ch = tid & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (h < RG) v = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(b) * a.Hq + g * RG + h) * kD) + ch);
+    *reinterpret_cast<uint4*>(qtile + h * 256 + ((ch ^ (h & 7)) << 4)) = v;
+  }
+  __syncthreads();   // (the first K / V tiles are already in flight)
+  const uint32_t q_row = smem_addr(qtile) + ((lm & 1) * 8 + lr) * 256;
   for (int tile = warp; tile < n_tiles; tile += NWARPS) {
     cp_async_wait<1>();   // this lane's K chunks of the tile
     __syncwarp();         // ... and every lane's
@@ -381,13 +405,15 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-#pragma unroll
+#pragma unroll 2
     for (int ks = 0; ks < kD / 16; ++ks) {
       uint32_t b0, b1, b2, b3;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(q_row + (static_cast<uint32_t>((2 * ks + (lm >> 1)) ^ lr) << 4), a0, a1, a2, a3);
       ldsm_x4(kb_s + ((lm >> 1) * 8 + lr) * 256 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4),
               b0, b1, b2, b3);
-      mma_bf16_16816(sacc[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-      mma_bf16_16816(sacc[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+      mma_bf16_16816(sacc[0], a0, a1, a2, a3, b0, b1);
+      mma_bf16_16816(sacc[1], a0, a1, a2, a3, b2, b3);
     }
     __syncwarp();
     issue(Ku, kbuf, tile + NWARPS);
@@ -466,28 +492,27 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
 
   constexpr int PS = part_stride(RG);
   float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * PS;
-  // thread (h, j): the 16 warp states of head h combined with weights
-  // e^(m_w - M), M the largest m_w (every thread of the head derives them)
-  for (int oi = tid; oi < RG * kD; oi += NT) {
-    const int h = oi / kD, j = oi % kD;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w) M = fmaxf(M, mer[(w * RG + h) * (kD + 2) + kD]);
-    float O = 0.f, L = 0.f;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w) {
-      const float* src = mer + (w * RG + h) * (kD + 2);
-      const float wgt = (M == -INFINITY) ? 0.f : exp2f(src[kD] - M);
-      O = fmaf(src[j], wgt, O);
-      L = fmaf(src[kD + 1], wgt, L);
-    }
-    if (a.C == 1) {
-      a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
-    } else {
-      part[h * (kD + 2) + j] = O;
-      if (j == 0) {
-        part[h * (kD + 2) + kD] = M;
-        part[h * (kD + 2) + kD + 1] = L;
+  {
+    // weights e^(m_w - M) of the 16 warp states of each head (warp h does
+    // head h), then thread (h, j) combines the outputs with them
+    float* wgt = mer + NWARPS * RG * (kD + 2);   // [RG][NWARPS]
+    float* hdr = wgt + NWARPS * RG;              // [RG][2]: M, sum of weighted l
+    if (warp < RG) merge_weights(mer + warp * (kD + 2), RG * (kD + 2), NWARPS, wgt + warp * NWARPS, hdr + 2 * warp);
+    __syncthreads();
+    for (int oi = tid; oi < RG * kD; oi += NT) {
+      const int h = oi / kD, j = oi % kD;
+      float O = 0.f;
+#pragma unroll 4
+      for (int w = 0; w < NWARPS; ++w) O = fmaf(mer[(w * RG + h) * (kD + 2) + j], wgt[h * NWARPS + w], O);
+      const float L = hdr[2 * h + 1];
+      if (a.C == 1) {
+        a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
+      } else {
+        part[h * (kD + 2) + j] = O;
+        if (j == 0) {
+          part[h * (kD + 2) + kD] = hdr[2 * h];
+          part[h * (kD + 2) + kD + 1] = L;
+        }
       }
     }
   }
@@ -509,20 +534,17 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
     for (int i = tid; i < n4; i += NT)
       reinterpret_cast<float4*>(sp)[i] = __ldcg(reinterpret_cast<const float4*>(parts) + i);
     __syncthreads();
+    float* wgt = sp + a.C * PS;   // [RG][C]
+    float* hdr = wgt + a.C * RG;  // [RG][2]
+    if (warp < RG) merge_weights(sp + warp * (kD + 2), PS, a.C, wgt + warp * a.C, hdr + 2 * warp);
+    __syncthreads();
     // thread (h, j): the C states of head h combined the same way
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
-      float M = -INFINITY;
-#pragma unroll 6
-      for (int cc = 0; cc < a.C; ++cc) M = fmaxf(M, sp[cc * PS + h * (kD + 2) + kD]);
-      float O = 0.f, L = 0.f;
-#pragma unroll 6
-      for (int cc = 0; cc < a.C; ++cc) {
-        const float* src = sp + cc * PS + h * (kD + 2);
-        const float wgt = (M == -INFINITY) ? 0.f : exp2f(src[kD] - M);
-        O = fmaf(src[j], wgt, O);
-        L = fmaf(src[kD + 1], wgt, L);
-      }
+      float O = 0.f;
+#pragma unroll 2
+      for (int cc = 0; cc < a.C; ++cc) O = fmaf(sp[cc * PS + h * (kD + 2) + j], wgt[h * a.C + cc], O);
+      const float L = hdr[2 * h + 1];
       a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
     }
   }
@@ -531,7 +553,7 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
 
 // ----------------------------------------------------------------------------
 template <int RG, int WORDS, int MODE>
-__global__ void __launch_bounds__(NT, 1) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_int[NWARPS + 16];
   __shared__ int s_aux[264];  // distance totals (<= 257 bins)

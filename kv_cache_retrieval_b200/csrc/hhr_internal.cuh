@@ -112,9 +112,10 @@ inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, 
     hist = sizeof(int) * ((size_t)C * (bits + 1) + 2 * (size_t)C) + 16;
   }
   if (mode != kModeSelect) {
-    const size_t ring = (size_t)(kDecodeThreads / 32) * 2 * 16 * 2 * kD;  // per warp: K and V of 16 tokens
+    // per warp: K and V of 16 tokens; then the 16-row query tile
+    const size_t ring = (size_t)(kDecodeThreads / 32) * 2 * 16 * 2 * kD + 16 * 2 * kD;
     size_t merge = sizeof(float) * ((kDecodeThreads / 32) * (size_t)r * (kD + 2) + (kDecodeThreads / 32) * (size_t)r + 2 * (size_t)r);
-    const size_t parts = sizeof(float) * ((size_t)C * part_stride(r) + (size_t)C * r + r);  // final merge
+    const size_t parts = sizeof(float) * ((size_t)C * part_stride(r) + (size_t)C * r + 2 * (size_t)r);  // final merge
     merge = merge > parts ? merge : parts;
     attn = ring > merge ? ring : merge;
   }
