@@ -522,6 +522,10 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   if (tid == 0) {
     const uint32_t old = atom_add_acq_rel(a.counters + unit, 1u);
     s_int[0] = (old == final_target - 1) ? 1 : 0;
+    // this CTA's share of the step is done but for the final merge: the
+    // next kernel on the stream may start launching (it waits for the
+    // completion of this one before touching memory)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
   __syncthreads();
   if (!s_int[0]) return;
@@ -555,6 +559,11 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
 template <int RG, int WORDS, int MODE>
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: wait here, before any global memory access, until that kernel
+  // has completed and its writes are visible.  Only the launch itself
+  // overlaps; no work of two steps does.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int s_int[NWARPS + 16];
   __shared__ int s_aux[264];  // distance totals (<= 257 bins)
   __shared__ float s_flt[4];
@@ -1283,6 +1292,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         if (tid == 0) {
           const uint32_t old = atom_add_acq_rel(ctr, 1u);
           if (old == 3u * a.C - 1u) atomicExch(ctr, 0u);
+          asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         }
       }
       __syncthreads();
@@ -1313,11 +1323,16 @@ cudaError_t launch_t(const DecodeArgs& a, size_t smem, cudaStream_t stream) {
   cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  // programmatic dependent launch: the kernel's CTAs may become resident
+  // while the previous kernel on the stream finishes (griddepcontrol.wait
+  // at the kernel's start keeps the two steps' work ordered)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
