@@ -220,7 +220,6 @@ __device__ bool unit_wait(const uint32_t* ctr, uint32_t target, const DecodeArgs
         ok = 0;
         break;
       }
-      __nanosleep(32);
     }
     *s_flag = ok;
   }
@@ -308,17 +307,24 @@ struct Smem {
 // State i has its running max at st[i * stride + d] and its sum at
 // st[i * stride + d + 1].  Writes wgt[i] = 2^(m_i - M) (M the largest m_i;
 // zero when every state is empty) and hdr = {M, sum_i wgt[i] l_i}.
+template <bool GLOBAL>
+__device__ __forceinline__ float state_ld(const float* p) {
+  if constexpr (GLOBAL) return __ldcg(p);   // written by other CTAs: read at L2
+  else return *p;
+}
+
+template <bool GLOBAL = false>
 __device__ __forceinline__ void merge_weights(const float* st, int stride, int n, float* wgt, float* hdr) {
   const int lane = threadIdx.x & 31;
   float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, st[i * stride + kD]);
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, state_ld<GLOBAL>(st + i * stride + kD));
 #pragma unroll
   for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
   float L = 0.f;
   for (int i = lane; i < n; i += 32) {
-    const float w = (M == -INFINITY) ? 0.f : exp2f(st[i * stride + kD] - M);
+    const float w = (M == -INFINITY) ? 0.f : exp2f(state_ld<GLOBAL>(st + i * stride + kD) - M);
     wgt[i] = w;
-    L = fmaf(st[i * stride + kD + 1], w, L);
+    L = fmaf(state_ld<GLOBAL>(st + i * stride + kD + 1), w, L);
   }
 #pragma unroll
   for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
@@ -530,24 +536,18 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   __syncthreads();
   if (!s_int[0]) return;
   if (a.C > 1) {
-    // all C partial states of the unit into shared memory in one pass
+    // the C partial states of the unit, read at L2: weights by one warp per
+    // head, then thread (h, j) combines column j of head h
     const float* parts = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit) * PS;
-    float* sp = reinterpret_cast<float*>(scratch);
-    const int n4 = a.C * PS / 4;
-#pragma unroll 8
-    for (int i = tid; i < n4; i += NT)
-      reinterpret_cast<float4*>(sp)[i] = __ldcg(reinterpret_cast<const float4*>(parts) + i);
+    float* wgt = reinterpret_cast<float*>(scratch);   // [RG][C]
+    float* hdr = wgt + a.C * RG;                      // [RG][2]
+    if (warp < RG) merge_weights<true>(parts + warp * (kD + 2), PS, a.C, wgt + warp * a.C, hdr + 2 * warp);
     __syncthreads();
-    float* wgt = sp + a.C * PS;   // [RG][C]
-    float* hdr = wgt + a.C * RG;  // [RG][2]
-    if (warp < RG) merge_weights(sp + warp * (kD + 2), PS, a.C, wgt + warp * a.C, hdr + 2 * warp);
-    __syncthreads();
-    // thread (h, j): the C states of head h combined the same way
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
       float O = 0.f;
-#pragma unroll 2
-      for (int cc = 0; cc < a.C; ++cc) O = fmaf(sp[cc * PS + h * (kD + 2) + j], wgt[h * a.C + cc], O);
+#pragma unroll 6
+      for (int cc = 0; cc < a.C; ++cc) O = fmaf(__ldcg(parts + cc * PS + h * (kD + 2) + j), wgt[h * a.C + cc], O);
       const float L = hdr[2 * h + 1];
       a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
     }
