@@ -3,12 +3,16 @@
 // One (sequence, KV head) pair -- a "unit" -- is spread over C CTAs of a
 // cooperative launch.  A fused step runs these phases per unit:
 //
-//   0  query prep      q~ = q R (Eq. 4) for the r query heads of the group
+//   0  query prep      R arrives by one bulk copy; q~ = q R (Eq. 4) for the
+//                      r query heads of the group, while every warp starts
+//                      streaming its own run of page metadata into a
+//                      lane-private shared-memory ring (cp.async, 16 B per
+//                      lane and page)
 //   1  page bounds     U_p = max_h sum_j max(q~_hj l_pj, q~_hj u_pj)  (Eq. 3)
-//                      over this CTA's contiguous slice of pages; metadata is
-//                      streamed with 128-bit loads, one page (512 B) per warp
-//                      load instruction, and the per-lane partial sums are
-//                      folded with a butterfly reduce-scatter
+//                      over this CTA's contiguous slice of pages, as a
+//                      tensor-core product of 16-page tiles of the stored
+//                      bounds with the exact bf16 terms of min(q~, 0) and
+//                      max(q~, 0); then the query codes (Eq. 10, sign) from W
 //      -- unit barrier 1 (U published in the workspace) --
 //   2  page top-P      every CTA reads all U of its unit and finds the same
 //                      P largest (ties to the lower page) with a 2048-bin
@@ -23,14 +27,16 @@
 //   5  token top-k     the histograms of all CTAs give the threshold distance
 //                      and each CTA's output offset; ties at the threshold go
 //                      to the lower token index across CTAs
-//   6  attention       each CTA attends over its own selected tokens: K/V rows
-//                      staged into shared memory with cp.async (16 B, L2 only),
-//                      one half-warp per token, online softmax in float32
+//   6  attention       each CTA attends over its own selected tokens in tiles
+//                      of 16 per warp on the tensor cores: K/V rows staged by
+//                      cp.async, online softmax in float32
 //      -- last-arriving CTA merges the C partial softmax states --
 //
-// Inter-CTA waits spin on workspace counters with a clock64() limit; on
-// expiry the kernel records HHR_ERR_TIMEOUT and returns.  The last CTA of a
-// unit resets its counter, so the workspace is zero again after each call.
+// The kernel is launched as a programmatic dependent of the previous kernel
+// on the stream and waits for it before touching memory.  Inter-CTA waits
+// spin on workspace counters with a clock64() limit; on expiry the kernel
+// records HHR_ERR_TIMEOUT and returns.  The last CTA of a unit resets its
+// counter, so the workspace is zero again after each call.
 
 #include <cuda_bf16.h>
 
