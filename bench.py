@@ -121,10 +121,15 @@ def encode_line(enc_ms, enc_flops, keys):
 
 
 def kernel_source_hash():
+    """Hash of the decode kernel's sources without comments and blank lines
+    (a comment edit does not invalidate a profile; any code change does)."""
     h = hashlib.sha256()
     for f in ("decode.cu", "hhr_internal.cuh"):
-        with open(os.path.join(ROOT, "kv_cache_retrieval_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "kv_cache_retrieval_b200", "csrc", f)) as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
