@@ -87,6 +87,29 @@ def algorithmic_bytes(w, n_valid, P, k):
     return parts, sum(parts.values())
 
 
+def planted_recall(tok_idx, n_sel, page_idx, planted_pos, page):
+    """Diagnostic, not a gate: the fraction of planted high-logit keys whose
+    token is selected, and whose page is kept, over all (sequence, KV head)
+    units.  tok_idx [B][Hkv][k], n_sel [B][Hkv], page_idx [B][Hkv][P] and
+    planted_pos [B][Hkv][m] are host arrays."""
+    import numpy as np
+    tok_hits = page_hits = total = 0
+    B, Hkv = n_sel.shape
+    for b in range(B):
+        for g in range(Hkv):
+            pl = planted_pos[b, g]
+            if pl.size == 0:
+                continue
+            sel = tok_idx[b, g, :max(int(n_sel[b, g]), 0)]
+            kept = page_idx[b, g][page_idx[b, g] >= 0]
+            tok_hits += int(np.isin(pl, sel).sum())
+            page_hits += int(np.isin(pl // page, kept).sum())
+            total += int(pl.size)
+    if total == 0:
+        return None
+    return {"tokens": round(tok_hits / total, 4), "pages": round(page_hits / total, 4), "planted": total}
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -380,6 +403,12 @@ def run_hhr(args):
     te1 = time.perf_counter()
     e2e_us = max_over_ranks((te1 - te0) * 1e6 / n_e2e, dev)
 
+    try:   # a diagnostic: it must not cost the bench line
+        recall = planted_recall(lay0["tok_idx"].cpu().numpy(), lay0["n_sel"].cpu().numpy(),
+                                lay0["page_idx"].cpu().numpy(), inp.planted_pos, w.page)
+    except Exception as exc:  # noqa: BLE001
+        recall = {"error": f"{type(exc).__name__}: {exc}"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, w, n_valid, args.cpu_seconds)
@@ -408,6 +437,7 @@ def run_hhr(args):
                     "d2h_bytes_per_step": int(out_pin.numel() * out_pin.element_size()),
                     "steps": n_e2e, "how": "pinned q H2D + hhr_decode_step + out D2H + sync, per step"},
             "gpu_launches": K,
+            "planted_recall": recall,
             "clocks": clocks,
             "encode": encode_line(enc_ms, enc_flops, w.B * w.Hkv * n_valid),
             "cpu_baseline": cpu,

@@ -47,3 +47,14 @@ def test_profile_hash_ignores_comments_only(tmp_path, monkeypatch):
     with open(csrc / "decode.cu", "a") as fh:
         fh.write("static int unused_symbol_for_the_test;\n")
     assert bench.kernel_source_hash() != h0
+
+
+def test_planted_recall_counts_selected_tokens_and_kept_pages():
+    import numpy as np
+    tok_idx = np.array([[[5, 17, 40, -1]]], np.int32)          # one unit, 3 selected
+    n_sel = np.array([[3]], np.int32)
+    page_idx = np.array([[[0, 2, -1]]], np.int32)               # pages of 16 tokens: 0..15, 32..47
+    planted = np.array([[[5, 20, 40, 47]]], np.int64)
+    r = bench.planted_recall(tok_idx, n_sel, page_idx, planted, 16)
+    assert r == {"tokens": 0.5, "pages": 0.75, "planted": 4}   # 5, 40 selected; 20 on page 1 (dropped)
+    assert bench.planted_recall(tok_idx, n_sel, page_idx, planted[:, :, :0], 16) is None
