@@ -376,6 +376,8 @@ def run_hhr(args):
 
     us_step = ms * 1000.0 / K
     keys_per_step = w.B * w.Hkv * n_valid
+    # tokens of the kept pages scored by Hamming distance in one step
+    candidates_per_step = w.B * w.Hkv * min(min(w.P, (n_valid + w.page - 1) // w.page) * w.page, n_valid)
     agg = aggregate(us_step, world, keys_per_step)
     parts, alg = algorithmic_bytes(w, n_valid, w.P, w.k)
     peak, peak_kind = measured_peak()
@@ -427,6 +429,7 @@ def run_hhr(args):
                 f"({alg * L / 2**20:.0f} MiB touched per cycle)", "launch": launch,
             },
             "keys_scored_per_s": agg["keys_scored_per_s"],
+            "candidates_scored_per_s": candidates_per_step * world / (us_step * 1e-6),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": profiled_traffic(w.name), "peak_source": peak_kind,
@@ -482,9 +485,32 @@ def cpu_baseline(inp, w, n_valid, seconds):
             break
     per_unit = (time.perf_counter() - t0) / n
     model, ncpu = host_info()
-    return {"value": round(per_unit * units * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+    line = {"value": round(per_unit * units * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"oracle decode of unit (0,0) of {units}, {n} runs in {seconds:.0f}s, "
                       f"scaled by {units}", "host_cpu": model, "host_nproc": ncpu}
+    try:   # the oracle's key encoding, timed on a bounded sample beside the decode step
+        line["encode"] = cpu_encode_baseline(inp, w, n_valid)
+    except Exception as exc:  # noqa: BLE001
+        line["encode"] = {"error": f"{type(exc).__name__}: {exc}"}
+    return line
+
+
+def cpu_encode_baseline(inp, w, n_valid, sample_keys=8192):
+    """The oracle's key encoding (rotation, page extrema, projection, codes)
+    of the first `sample_keys` keys of unit (0, 0), single-threaded, scaled to
+    all keys of all units."""
+    import numpy as np
+    from oracle import oracle as O
+    n = min(sample_keys, n_valid)
+    codes = np.zeros((w.n_cap, w.words), np.uint32)
+    meta = np.zeros((w.np_cap, 2, w.d), np.uint16)
+    K = np.ascontiguousarray(inp.K[0, 0])
+    t0 = time.perf_counter()
+    O.encode_unit(K, 0, n, w.page, inp.R[0], inp.W[0], codes, meta)
+    dt = time.perf_counter() - t0
+    units = w.B * w.Hkv
+    return {"ms": round(dt * (n_valid / max(n, 1)) * units * 1e3, 1), "cores": 1,
+            "sample": f"oracle encoding of {n} keys of unit (0,0), scaled to {n_valid} keys x {units} units"}
 
 
 def run_reference(args):
