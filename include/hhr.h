@@ -37,6 +37,10 @@
  *     returns.
  *   Streams.  `stream` is a cudaStream_t (NULL: the legacy default stream).
  *     Device work is enqueued on it and the call returns without waiting.
+ *     The decode kernels are launched as programmatic dependents of the
+ *     preceding kernel on the stream: they may become resident early but
+ *     wait for that kernel's completion before touching memory, so stream
+ *     order is kept.
  *   Errors.  Every call returns an hhr_status.  Arguments are checked on the
  *     host first; on any return other than HHR_OK or HHR_ERR_CUDA nothing was
  *     enqueued.  HHR_ERR_CUDA reports a failed launch (cudaGetLastError).
