@@ -305,7 +305,7 @@ def run_hhr(args):
         lay = dict(
             K=K0 if li == 0 else K0.clone(), V=V0 if li == 0 else V0.clone(),
             codes=codes0 if li == 0 else codes0.clone(), meta=meta0 if li == 0 else meta0.clone(),
-            q=q_dev.clone(),
+            q=q_dev.clone(), R=R if li == 0 else R.clone(), W=W if li == 0 else W.clone(),
             page_idx=torch.empty(w.B, w.Hkv, w.P, dtype=torch.int32, device=dev),
             tok_idx=torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=dev),
             n_sel=torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev),
@@ -315,7 +315,7 @@ def run_hhr(args):
     scale = 1.0 / math.sqrt(w.d)
 
     def step(lay, stream=None):
-        hhr.hhr_decode_step(dims, lay["q"], R, W, lay["codes"], lay["meta"], lay["K"], lay["V"],
+        hhr.hhr_decode_step(dims, lay["q"], lay["R"], lay["W"], lay["codes"], lay["meta"], lay["K"], lay["V"],
                             n_valid, w.P, w.k, scale, lay["page_idx"], lay["tok_idx"], lay["n_sel"],
                             lay["out"], ws, None, stream)
 
