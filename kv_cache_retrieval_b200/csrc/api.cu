@@ -88,60 +88,31 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   int C = resident / units;
   if (C < 1) C = 1;
   if (C > kMaxCtasPerUnit) C = kMaxCtasPerUnit;
-  int slice_pages = 0, slice_tokens = 0;
   if (mode == kModeAttend) {
     const int by_tokens = (k + 63) / 64;  // at least 64 tokens per CTA
     if (C > by_tokens) C = by_tokens < 1 ? 1 : by_tokens;
-    for (;;) {
-      slice_tokens = (k + C - 1) / C + 1;
-      if (slice_tokens <= kMaxTokensPerCta || C >= kMaxCtasPerUnit || C >= resident) break;
-      ++C;
-    }
   } else {
     const int by_pages = (NP + kMinPagesPerCta - 1) / kMinPagesPerCta;
     if (C > by_pages) C = by_pages < 1 ? 1 : by_pages;
-    for (;;) {
-      slice_pages = (NP + C - 1) / C;
-      // a CTA ranks the tokens of its own kept pages
-      slice_tokens = (slice_pages < Pk ? slice_pages : Pk) * d->page;
-      if ((slice_pages <= kMaxSlicePages && slice_tokens <= kMaxTokensPerCta) ||
-          C >= kMaxCtasPerUnit || C >= resident)
-        break;
-      ++C;
+  }
+  int slice_pages = 0, slice_tokens = 0;
+  for (;;) {
+    if (mode == kModeAttend) {
+      slice_pages = 0;
+      slice_tokens = (k + C - 1) / C + 1;
+    } else {
+      slice_pages = (Pk + C - 1) / C;
+      slice_tokens = slice_pages * d->page;
     }
-    if (slice_pages > kMaxSlicePages) return HHR_ERR_UNSUPPORTED;
+    if (slice_tokens <= kMaxTokensPerCta || C >= kMaxCtasPerUnit || C * units >= resident) break;
+    ++C;
   }
   if (slice_tokens > kMaxTokensPerCta) return HHR_ERR_UNSUPPORTED;
-  const DecodeSmem lay = decode_smem(r, d->bits, slice_pages, mode);
+  const DecodeSmem lay = decode_smem(NP, C, d->bits, r, slice_pages, slice_tokens, mode);
   if (lay.total > info.smem_optin) return HHR_ERR_UNSUPPORTED;
   int grid_units = resident / C;
   if (grid_units > units) grid_units = units;
   if (grid_units < 1) grid_units = 1;
-
-  // page exchange: units of few pages (or one CTA) score every page in
-  // every CTA; larger ones bin their own pages by a common sample
-  const bool local = mode != kModeAttend && (NP <= kLocalMaxPages || C == 1);
-  int n_sample = 0, b_exp = 0, win = 0;
-  if (mode != kModeAttend) {
-    if (local) {
-      n_sample = C == 1 ? 0 : NP;
-    } else {
-      n_sample = kSample;
-      b_exp = static_cast<int>(static_cast<long long>(Pk) * kSample / NP);
-      if (b_exp > kSample) b_exp = kSample;
-      // about six bins' worth of each CTA's entries on either side of the
-      // expected cutoff, within the ring
-      const long long per_bin = (static_cast<long long>(NP) + static_cast<long long>(kSample) * C - 1) /
-                                (static_cast<long long>(kSample) * C);
-      long long w = 6 * per_bin;
-      if (w < 16) w = 16;
-      if (w > kWinMax) w = kWinMax;
-      win = static_cast<int>((w + 1) / 2 * 2);
-      const size_t cum_bytes = align_up(sizeof(int) * static_cast<size_t>(C) * (kSample + 2), 16);
-      while (win > 2 && cum_bytes + static_cast<size_t>(C) * 2 * win * 8 > static_cast<size_t>(kRingBytes))
-        win -= 2;
-    }
-  }
 
   a->B = d->B;
   a->Hq = d->Hq;
@@ -159,13 +130,7 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   a->grid_units = grid_units;
   a->slice_pages = slice_pages;
   a->slice_tokens = slice_tokens;
-  a->local = local ? 1 : 0;
-  a->n_sample = n_sample;
-  a->b_exp = b_exp;
-  a->win = win;
-  a->list_half = (slice_pages + 1) / 2 * 2;
   a->spin_limit = kSpinLimit;
-  a->test_extra_stage = 0;
   *smem = lay.total;
   return HHR_OK;
 }
@@ -175,12 +140,11 @@ void carve_workspace(void* ws, const hhr_dims* d, DecodeArgs* a) {
   unsigned char* base = static_cast<unsigned char*>(ws);
   a->status = reinterpret_cast<uint32_t*>(base + L.status);
   a->counters = reinterpret_cast<uint32_t*>(base + L.counters);
-  a->wsCum = reinterpret_cast<int32_t*>(base + L.cum);
-  a->wsList = reinterpret_cast<int2*>(base + L.list);
-  a->wsCumD = reinterpret_cast<int32_t*>(base + L.cumD);
+  a->wsU = reinterpret_cast<float*>(base + L.U);
+  a->wsMinMax = reinterpret_cast<float*>(base + L.minmax);
+  a->wsHist = reinterpret_cast<int32_t*>(base + L.hist);
   a->wsPart = reinterpret_cast<float*>(base + L.part);
-  a->list_stride = L.list_stride;
-  a->cumD_stride = L.cumD_stride;
+  a->np_stride = L.np_stride;
 }
 
 int32_t check_workspace(const hhr_dims* d, void* ws, size_t ws_bytes) {
@@ -257,11 +221,11 @@ static int32_t decode_common(const hhr_dims* dims, int mode, const void* q, cons
                              int32_t* dbg_D, void* workspace, size_t ws_bytes, void* stream) {
   if (int32_t st = check_dims(dims)) return st;
   if (np_cap_of(dims) > HHR_MAX_PAGES) return HHR_ERR_UNSUPPORTED;
-  if (k < 1 || !q || !aligned16(q)) return HHR_ERR_INVALID_ARG;
+  if (k < 1 || !q) return HHR_ERR_INVALID_ARG;
   if (mode != kModeAttend) {
     if (P < 1 || n_valid < 0 || n_valid > dims->n_cap) return HHR_ERR_INVALID_ARG;
     if (!R || !W || !codes || !meta || !page_idx || !tok_idx || !n_sel) return HHR_ERR_INVALID_ARG;
-    if (!aligned16(codes) || !aligned16(meta) || !aligned16(R) || !aligned16(W)) return HHR_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(meta)) return HHR_ERR_INVALID_ARG;
   }
   if (mode != kModeSelect) {
     if (!K || !V || !out) return HHR_ERR_INVALID_ARG;

@@ -1,42 +1,36 @@
 // Decode-time retrieval kernels for sm_100a.
 //
 // One (sequence, KV head) pair -- a "unit" -- is spread over C CTAs of a
-// cooperative launch; CTA c owns the contiguous page range [c NP / C,
-// (c + 1) NP / C).  A fused step runs these phases per unit:
+// cooperative launch.  A fused step runs these phases per unit:
 //
-//   0  query prep      R arrives by one bulk copy while the metadata ring
-//                      fills; q~ = q R (Eq. 4) for the r query heads
-//   1  page bounds     U_p = max_h sum_j max(q~_hj l_pj, q~_hj u_pj) (Eq. 3)
-//                      for a common sample of the unit's pages and for the
-//                      CTA's own pages.  The metadata streams through a ring
-//                      of 16-KiB bulk copies (the warp that frees a slot
-//                      refills it); warps score 8-page tasks with packed
-//                      float32 FMAs and a butterfly reduction
-//   2  publish         every CTA sorts the sample (identically), bins its own
-//                      bounds by the sample values, publishes its cumulative
-//                      bin counts and its bounds ordered by bin, and arrives
-//                      at unit barrier 1; then forms the query codes (Eq. 10,
-//                      sign) from W
-//      -- unit barrier 1 --
-//   3  page top-P      one read of every CTA's counts and of the stretch of
-//                      its list around the expected cutoff bin gives the
-//                      boundary bin, and an exact ranking of that bin's
-//                      entries gives the cutoff (bound, page): a page is kept
-//                      iff (U, -page) is not below it, ties to the lower page
+//   0  query prep      R arrives by one bulk copy; q~ = q R (Eq. 4) for the
+//                      r query heads of the group, while every warp starts
+//                      streaming its own run of page metadata into a
+//                      lane-private shared-memory ring (cp.async, 16 B per
+//                      lane and page)
+//   1  page bounds     U_p = max_h sum_j max(q~_hj l_pj, q~_hj u_pj)  (Eq. 3)
+//                      over this CTA's contiguous slice of pages, as a
+//                      tensor-core product of 16-page tiles of the stored
+//                      bounds with the exact bf16 terms of min(q~, 0) and
+//                      max(q~, 0); then the query codes (Eq. 10, sign) from W
+//      -- unit barrier 1 (U published in the workspace) --
+//   2  page top-P      every CTA reads all U of its unit and finds the same
+//                      P largest (ties to the lower page) with a 2048-bin
+//                      histogram over [min U, max U] plus an exact ranking of
+//                      the boundary bin
+//   3  compaction      kept pages in ascending order; CTA c takes the c-th
+//                      slice of them
 //   4  Hamming         D_n = min_h popc(qcode_h xor code_n) (Eq. 2) for the
-//                      tokens of the CTA's own kept pages; the cumulative
-//                      histogram of D is published
+//                      tokens of the slice, one 16/32-B code load per token;
+//                      a (b+1)-bin histogram of D is published
 //      -- unit barrier 2 --
-//   5  token top-k     the histograms of all CTAs give the threshold distance,
-//                      each CTA's quota of threshold ties (lower tokens first)
-//                      and its output offset
-//   6  attention       softmax(scale q.k) v over the CTA's selected tokens:
-//                      K/V rows by bulk copy into per-warp double buffers,
-//                      float32 dot products and online softmax
-//      -- the last-arriving CTA merges the C partial softmax states --
-//
-// Units with at most kLocalMaxPages pages, or with a single CTA, skip the
-// exchange of phase 3: every CTA scores every page.
+//   5  token top-k     the histograms of all CTAs give the threshold distance
+//                      and each CTA's output offset; ties at the threshold go
+//                      to the lower token index across CTAs
+//   6  attention       each CTA attends over its own selected tokens in tiles
+//                      of 16 per warp on the tensor cores: K/V rows staged by
+//                      cp.async, online softmax in float32
+//      -- last-arriving CTA merges the C partial softmax states --
 //
 // The kernel is launched as a programmatic dependent of the previous kernel
 // on the stream and waits for it before touching memory.  Inter-CTA waits
@@ -47,7 +41,6 @@
 #include <cuda_bf16.h>
 
 #include <cfloat>
-#include <climits>
 #include <cstdint>
 
 #include "hhr_internal.cuh"
@@ -57,14 +50,7 @@ namespace {
 
 constexpr int NT = kDecodeThreads;
 constexpr int NWARPS = NT / 32;
-constexpr unsigned FULL = 0xFFFFFFFFu;
-constexpr int kTaskPages = 8;                              // pages one warp scores per task
-constexpr int kTasksPerChunk = kChunkPages / kTaskPages;   // 4
-static_assert(NT == 4 * kD, "query products use four row quarters of 128 columns");
-static_assert(kSlots * kChunkBytes == kRingBytes, "ring size");
-static_assert(NWARPS * 8192 <= kRingBytes, "per-warp K/V double buffers live in the ring");
 
-// ------------------------------------------------------------ PTX helpers
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
@@ -78,20 +64,21 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
   return old;
 }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(d), "l"(gmem_src) : "memory");
+}
+// Copies 16 B when src_bytes is 16, writes 16 zero bytes when it is 0.
+__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(d), "l"(gmem_src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// CTA-scope acquire-release add on a shared-memory word.
-__device__ __forceinline__ uint32_t smem_atom_add_acq_rel(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
-               : "=r"(old) : "r"(smem_addr(p)), "r"(v) : "memory");
-  return old;
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -104,46 +91,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 
 // 1-D bulk copy global -> shared on the TMA unit; completion is signalled on
 // the mbarrier as transferred bytes.  Both addresses 16-B aligned, size a
-// multiple of 16.  This GPU's memory only; no multicast.
+// multiple of 16.  No multicast.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
-
-// The same copy with an L2 cache policy (createpolicy): evict-last for the
-// small tensors every step re-reads (R, W).
-__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
-                                              uint64_t policy) {
+// The same copy with an L2 cache policy: evict-last for the small tensors
+// every step re-reads (R, W).
+__device__ __forceinline__ void bulk_g2s_keep(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
-               :: "r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(policy) : "memory");
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-// Copies `rows` rows of `chunks` 16-B chunks from global (row stride
-// src_stride bytes, read at L2) to shared memory (row stride dst_stride
-// bytes) with cp.async; warp w takes rows w, w + 16, ...  Chunks whose index
-// is outside [c_lo, c_hi) are skipped.  Commits one group; the caller waits
-// (cp_async_wait<0>) and synchronises.
-__device__ __forceinline__ void copy_rows_async(uint32_t dst, const char* src, int rows, int chunks,
-                                                size_t src_stride, uint32_t dst_stride, int c_lo, int c_hi) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int r = warp; r < rows; r += NT / 32)
-    for (int ch = lane; ch < chunks; ch += 32)
-      if (ch >= c_lo && ch < c_hi)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                     :: "r"(dst + r * dst_stride + ch * 16), "l"(src + r * src_stride + ch * 16) : "memory");
-  asm volatile("cp.async.commit_group;" ::: "memory");
+               :: "r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(pol) : "memory");
 }
 
 // Brings the 128-B line holding `p` into L2 (no register result).
@@ -169,32 +129,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   return false;
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-
-// The two bf16 halves of a word, widened exactly to float32.
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// ------------------------------------------------------- block primitives
-
 // Exclusive prefix sum over the CTA.  Every thread must call it.
 __device__ int block_excl_scan(int v, int* s_warp, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(FULL, x, o);
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
     if (lane >= o) x += y;
   }
   if (lane == 31) s_warp[warp] = x;
@@ -204,7 +145,7 @@ __device__ int block_excl_scan(int v, int* s_warp, int* total) {
     int wx = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(FULL, wx, o);
+      const int y = __shfl_up_sync(0xFFFFFFFFu, wx, o);
       if (lane >= o) wx += y;
     }
     if (lane < NWARPS) s_warp[lane] = wx - w;
@@ -225,7 +166,7 @@ __device__ __forceinline__ int block_excl_scan1(int v, int* s_warp, int* total) 
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(FULL, x, o);
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
     if (lane >= o) x += y;
   }
   if (lane == 31) s_warp[warp] = x;
@@ -247,219 +188,89 @@ __device__ int block_sum(int v, int* s_warp) {
   return total;
 }
 
-// Order-preserving map of a float to uint32 (-0 and +0 map together).
 __device__ __forceinline__ uint32_t order_key(float u) {
-  const uint32_t x = __float_as_uint(u + 0.0f);
+  const uint32_t x = __float_as_uint(u + 0.0f);  // -0 -> +0
   return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
 }
 
-// ------------------------------------------------- page cutoff (top-P)
-//
-// The kept pages are the Pk largest in the order (bound descending, page
-// ascending).  The cutoff is the Pk-th element of that order: a page is kept
-// iff (key, page) is not below it, i.e. key > pk.key, or key == pk.key and
-// page <= pk.page.
-struct Pivot {
-  uint32_t key;
-  int page;
-  int all;  // every candidate is kept
-};
-
-__device__ __forceinline__ bool kept(uint32_t key, int page, const Pivot& pv) {
-  return pv.all || key > pv.key || (key == pv.key && page <= pv.page);
-}
-
-// The need-th element by exact bitwise search: the need-th largest key, then
-// the page among that key's entries.  For very many equal-looking bounds;
-// kept out of line.
-__device__ __noinline__ Pivot select_pivot_bitwise(const float* vals, const int* ids, int id0, int M,
-                                                  int need, int* s_scan) {
+// Exact top-`Pk` of the NP bounds in sU, ties to the lower page index, as a
+// bitmap: a 32-step bitwise search for the Pk-th largest order key, then a
+// page-order scan for the ties.  Used only when very many bounds fall into
+// one histogram bin (degenerate inputs), so it is kept out of line.
+__device__ __noinline__ void exact_top_pages(const float* sU, int NP, int Pk, int* s_scan,
+                                             uint32_t* sBits) {
   const int tid = threadIdx.x;
-  auto id_of = [&](int i) { return ids ? ids[i] : id0 + i; };
   uint32_t T = 0u;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
     int cnt = 0;
-    for (int i = tid; i < M; i += NT) cnt += order_key(vals[i]) >= cand;
-    if (block_sum(cnt, s_scan) >= need) T = cand;
+    for (int p = tid; p < NP; p += NT) cnt += order_key(sU[p]) >= cand;
+    if (block_sum(cnt, s_scan) >= Pk) T = cand;
   }
   int gt = 0;
-  for (int i = tid; i < M; i += NT) gt += order_key(vals[i]) > T;
-  const int r = need - block_sum(gt, s_scan);   // >= 1
-  int X = 0;                                   // the r-th smallest page with key T
-  for (int bit = 14; bit >= 0; --bit) {
-    const int cand = X | (1 << bit);
-    int cnt = 0;
-    for (int i = tid; i < M; i += NT) cnt += (order_key(vals[i]) == T) && (id_of(i) < cand);
-    if (block_sum(cnt, s_scan) < r) X = cand;
+  for (int p = tid; p < NP; p += NT) gt += order_key(sU[p]) > T;
+  const int need_eq = Pk - block_sum(gt, s_scan);
+  const int span = (NP + NT - 1) / NT;
+  const int lo = tid * span, hi = min(NP, lo + span);
+  int eq = 0;
+  for (int p = lo; p < hi; ++p) eq += order_key(sU[p]) == T;
+  int eqtot;
+  int er = block_excl_scan(eq, s_scan, &eqtot);
+  for (int p = lo; p < hi; ++p) {
+    const uint32_t kk = order_key(sU[p]);
+    bool keep = kk > T;
+    if (kk == T) keep = (er++ < need_eq);
+    if (keep) atomicOr(&sBits[p >> 5], 1u << (p & 31));
   }
-  Pivot pv;
-  pv.all = 0;
-  pv.key = T;
-  pv.page = X;
-  return pv;
 }
 
-// (bound order key, page) as one 64-bit value whose unsigned order is the
-// selection order: larger bound first, then lower page.
-__device__ __forceinline__ unsigned long long lex_key(uint32_t key, int page) {
-  return (static_cast<unsigned long long>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(page));
-}
-
-// The entry of rank nd - 1 (0-based, largest first) among n <= kRankMax
-// distinct lexicographic keys lk[0..n): its key is counted against the
-// others by NT / n_pow2 threads over slices and summed in shared memory
-// (n <= 32: one warp, no block barrier before the result).  The winner is
-// written to *win; every thread calls it and sees *win afterwards.
-constexpr int kRankMax = 512;
-__device__ void rank_lex(const unsigned long long* lk, int n, int nd, int* rk, unsigned long long* win) {
-  const int tid = threadIdx.x;
-  if (n <= 32) {
-    if (tid < 32) {
-      const unsigned long long ki = tid < n ? lk[tid] : 0ull;
-      int r = 0;
-      for (int j = 0; j < n; ++j) r += lk[j] > ki;
-      if (tid < n && r == nd - 1) *win = ki;
+// For a histogram of kBuckets bins and a count `need` >= 1 not above its
+// total, finds the bin b* holding the need-th largest element (bins ordered
+// by value) and the number of elements in bins above b*.  Thread t owns the
+// four bins [4(NT-1-t), 4(NT-1-t) + 4), so a scan in thread order counts the
+// elements in higher bins.  Every thread must call it; results in out[0..1].
+__device__ void find_boundary(const int* hist, int need, int* s_warp, int* out) {
+  static_assert(kBuckets == 4 * NT, "bin ownership assumes 4 bins per thread");
+  const int base = 4 * (NT - 1 - static_cast<int>(threadIdx.x));
+  const int c4 = hist[base] + hist[base + 1] + hist[base + 2] + hist[base + 3];
+  int tot;
+  int running = block_excl_scan(c4, s_warp, &tot);
+  for (int bin = base + 3; bin >= base; --bin) {
+    const int hcount = hist[bin];
+    if (running < need && running + hcount >= need) {
+      out[0] = bin;
+      out[1] = running;
     }
-    __syncthreads();
-    return;
+    running += hcount;
   }
-  int np2 = 64;
-  while (np2 < n) np2 <<= 1;               // <= kRankMax
-  const int parts = NT / np2;              // threads per entry
-  if (tid < np2) rk[tid] = 0;
-  __syncthreads();
-  {
-    const int i = tid % np2, part = tid / np2;
-    if (i < n) {
-      const unsigned long long ki = lk[i];
-      const int j0 = part * n / parts, j1 = (part + 1) * n / parts;
-      int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
-      int j = j0;
-      for (; j + 3 < j1; j += 4) {
-        r0 += lk[j] > ki;
-        r1 += lk[j + 1] > ki;
-        r2 += lk[j + 2] > ki;
-        r3 += lk[j + 3] > ki;
-      }
-      for (; j < j1; ++j) r0 += lk[j] > ki;
-      atomicAdd(&rk[i], (r0 + r1) + (r2 + r3));
-    }
-  }
-  __syncthreads();
-  if (tid < n && rk[tid] == nd - 1) *win = lk[tid];
   __syncthreads();
 }
 
-constexpr int kSubBins = 64;   // linear bins over a candidate set's value range
-
-// The need-th element (1 <= need <= M) of entries i < M in the order (bound
-// descending, page ascending); the bound of entry i is vals[i], its page
-// ids[i] (or id0 + i when ids is null).  Pages are distinct and below 2^15.
-// Up to kRankMax entries are ranked directly.  Larger sets are first cut
-// down by linear bins over [min, max] of the bounds to the bin holding the
-// need-th element (a bitwise search over all entries when very many bounds
-// fall into one bin, e.g. equal bounds).  `scratch` holds at least
-// kSubBins + 3 kRankMax ints.  Every thread must call it; every thread gets
-// the same result.
-__device__ Pivot select_pivot(const float* vals, const int* ids, int id0, int M, int need,
-                              int* scratch, int* s_scan, int* s_misc, float* s_flt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  auto id_of = [&](int i) { return ids ? ids[i] : id0 + i; };
-  int* hist = scratch;                                                                 // [kSubBins]
-  unsigned long long* lk = reinterpret_cast<unsigned long long*>(scratch + kSubBins);  // [kRankMax]
-  int* rk = scratch + kSubBins + 2 * kRankMax;                                         // [kRankMax]
-  __shared__ unsigned long long s_win;
-  Pivot pv;
-  pv.all = 0;
-  if (M <= kRankMax) {
-    for (int i = tid; i < M; i += NT) lk[i] = lex_key(order_key(vals[i]), id_of(i));
-    __syncthreads();
-    rank_lex(lk, M, need, rk, &s_win);
-    pv.key = static_cast<uint32_t>(s_win >> 32);
-    pv.page = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(s_win));
-    __syncthreads();
-    return pv;
-  }
-  float mn = INFINITY, mx = -INFINITY;
-  for (int i = tid; i < M; i += NT) {
-    mn = fminf(mn, vals[i]);
-    mx = fmaxf(mx, vals[i]);
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-  }
-  if (lane == 0) {
-    s_flt[2 * warp] = mn;
-    s_flt[2 * warp + 1] = mx;
-  }
-  if (tid < kSubBins) hist[tid] = 0;
-  if (tid == 0) s_misc[4] = 0;
-  __syncthreads();
-  mn = INFINITY;
-  mx = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < NWARPS; ++w) {
-    mn = fminf(mn, s_flt[2 * w]);
-    mx = fmaxf(mx, s_flt[2 * w + 1]);
-  }
-  const float range = mx - mn;
-  const float inv = (range > 0.f && range <= FLT_MAX) ? static_cast<float>(kSubBins) / range : 0.f;
-  // bin = round((u - mn) * inv) by one FMA (the 1.5 * 2^23 offset leaves the
-  // rounded integer in the low mantissa bits); monotone in u, clamped.
-  auto bucket = [&](float u) {
-    const int bk = __float_as_int(fmaf(u - mn, inv, 12582912.f)) - 0x4B400000;
-    return min(max(bk, 0), kSubBins - 1);
-  };
-  for (int i = tid; i < M; i += NT) atomicAdd(&hist[bucket(vals[i])], 1);
-  __syncthreads();
-  if (warp == 0) {   // from the top bin down: the bin holding the need-th element
-    const int b0 = kSubBins - 1 - 2 * lane, b1 = b0 - 1;   // lane owns two bins, higher first
-    const int h0 = hist[b0], h1 = hist[b1];
-    int x = h0 + h1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(FULL, x, o);
-      if (lane >= o) x += y;
-    }
-    const int before = x - h0 - h1;   // entries in higher bins than b0
-    if (before < need && before + h0 >= need) {
-      s_misc[2] = b0;
-      s_misc[3] = before;
-    } else if (before + h0 < need && before + h0 + h1 >= need) {
-      s_misc[2] = b1;
-      s_misc[3] = before + h0;
-    }
-  }
-  __syncthreads();
-  const int b2 = s_misc[2];
-  const int need2 = need - s_misc[3];
-  const int n2 = hist[b2];
-  if (n2 <= kRankMax) {
-    for (int i = tid; i < M; i += NT) {
-      if (bucket(vals[i]) == b2) {
-        const int slot = atomicAdd(&s_misc[4], 1);
-        lk[slot] = lex_key(order_key(vals[i]), id_of(i));
+// Thread 0 waits until the unit counter reaches `target` (acquire), then the
+// CTA barrier releases everyone.  Returns false (HHR_ERR_TIMEOUT recorded)
+// if the wait ran out.  Every thread of the CTA calls it.
+__device__ bool unit_wait(const uint32_t* ctr, uint32_t target, const DecodeArgs& a, int* s_flag) {
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const long long t0 = clock64();
+    while (ld_acquire(ctr) < target) {
+      if (static_cast<unsigned long long>(clock64() - t0) > a.spin_limit) {
+        atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+        ok = 0;
+        break;
       }
     }
-    __syncthreads();
-    rank_lex(lk, n2, need2, rk, &s_win);
-    pv.key = static_cast<uint32_t>(s_win >> 32);
-    pv.page = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(s_win));
-    __syncthreads();
-    return pv;
+    *s_flag = ok;
   }
-  return select_pivot_bitwise(vals, ids, id0, M, need, s_scan);
+  __syncthreads();
+  return *s_flag != 0;
 }
-
-// ------------------------------------------------------------ query prep
 
 // x[r][d] . M[d][d] (both float32 in shared memory), in eight row groups:
 // thread t forms, for every head h, the partial sums over rows
 // [16 (t / 64), 16 (t / 64) + 16) of columns 2 (t % 64) and 2 (t % 64) + 1
-// (packed FMAs).  M is read once per CTA, conflict-free; x by broadcast.
+// with packed float32 FMAs.  M is read once per CTA, conflict-free; x by
+// broadcast.
 template <int RG>
 __device__ __forceinline__ void product_partials(const float* x, const float* M, float2 (&acc)[RG]) {
   static_assert(NT == 8 * 64, "eight row groups of 64 column pairs");
@@ -502,357 +313,256 @@ __device__ __forceinline__ float product_sum(const float* part, int oi) {
   return s0 + s1;
 }
 
-// res[h * kD + j] = (x . M)[h][j] for the r query heads; M (64 KiB) is
-// overwritten by the partial sums.  Every thread calls it.
-template <int RG>
-__device__ void query_product(const float* x, float* M, float* res) {
-  float2 acc[RG];
-  product_partials<RG>(x, M, acc);
-  __syncthreads();                           // every thread has read M
-  store_partials<RG>(acc, M);
-  __syncthreads();
-  for (int oi = threadIdx.x; oi < RG * kD; oi += NT) res[oi] = product_sum<RG>(M, oi);
-  __syncthreads();
+// ldmatrix: four (two) 8x8 b16 matrices; lane i supplies the row address of
+// matrix i / 8, row i % 8 (lanes 0-15 for x2).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
 }
 
-// ----------------------------------------------------- page bounds (Eq. 3)
-//
-// A warp scores 8 pages per task.  With HG heads per pass, LPP = 4 HG lanes
-// share a page: lane j of the group holds dims [8 (j NCH + c), + 8) for its
-// NCH = 4 / HG chunks c of the lower and the upper row (16 B each), so a
-// page's bound is a sum over LPP lanes of per-lane partials.  The pair
-// (l_d, u_d) times (min(q~_hd, 0), max(q~_hd, 0)) is one packed FMA, which is
-// max(q~ l, q~ u) summed over the pair.  The chunk order is rotated per lane
-// so that a quarter-warp's 16-B loads hit distinct banks.
-template <int HG>
-struct BoundsLayout {
-  static constexpr int LPP = 4 * HG;            // lanes per page
-  static constexpr int NCH = 4 / HG;            // 16-B chunks per row and lane
-  static constexpr int PPS = 32 / LPP;          // pages per warp step
-  static constexpr int STEPS = kTaskPages / PPS;  // == HG
-  static constexpr int NV = STEPS * HG;         // partials per lane before reduction
+// d += A (16 x 16, row-major bf16) * B (16 x 8, column-major bf16), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+               "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// v = hi + mid + lo exactly, each term a bf16 (v - hi and the next residual
+// are exact in float32, and the last residual has at most 8 significant
+// bits).  Stores the terms at column k of rows n0, n0 + 1, n0 + 2 of the
+// [rows][256] bf16 operand whose 16-B chunks are swizzled by row & 7.
+__device__ __forceinline__ void put_terms(uint16_t* qb, int n0, int k, float v) {
+  float rest = v;
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    const __nv_bfloat16 term = __float2bfloat16_rn(rest);
+    rest -= __bfloat162float(term);
+    const int n = n0 + t;
+    qb[n * (2 * kD) + (((k >> 3) ^ (n & 7)) << 3) + (k & 7)] = __bfloat16_as_ushort(term);
+  }
+}
+
+struct Smem {
+  uint16_t* qb;    // bf16 terms of [min(q~, 0) ; max(q~, 0)], [8 nb][2 d], 16-B chunks swizzled
+  float* qf;       // [r][d] queries (float), pre-scaled for attention
+  uint32_t* qc;    // [r][w] query codes
+  int* my_pages;   // kept pages of this CTA's slice
+  uint16_t* tokD;  // distances of the slice's tokens
+  int* sel;        // selected tokens of this CTA (ascending)
+  unsigned char* scratch;
 };
 
-// Butterfly reduce-scatter of NV values over groups of LPP lanes: afterwards
-// v[0] holds the group sum of one value index (see the callers).
-template <int NV, int O>
-struct ReduceScatter {
-  static __device__ __forceinline__ void run(float* v, int lane) {
-    if constexpr (NV > 1) {
-      constexpr int H = NV / 2;
-      const bool up = (lane & O) != 0;
-#pragma unroll
-      for (int i = 0; i < H; ++i) {
-        const float send = up ? v[i] : v[i + H];
-        const float keep = up ? v[i + H] : v[i];
-        v[i] = keep + __shfl_xor_sync(FULL, send, O);
-      }
-      if constexpr (O > 1) ReduceScatter<H, O / 2>::run(v, lane);
-    } else {
-      v[0] += __shfl_xor_sync(FULL, v[0], O);
-      if constexpr (O > 1) ReduceScatter<1, O / 2>::run(v, lane);
-    }
-  }
-};
-
-// Loads this lane's (min(q~,0), max(q~,0)) pairs for heads [h0, h0 + HG).
-template <int HG>
-__device__ __forceinline__ void load_qpairs(const float* qt, int h0, float2 (&qp)[32], int lane) {
-  using L = BoundsLayout<HG>;
-  const int j = lane % L::LPP;
-  const int rot = ((lane & 7) * L::NCH) >> 3;
-#pragma unroll
-  for (int i = 0; i < L::NCH; ++i) {
-    const int c = (i + rot) % L::NCH;
-    const int d0 = 8 * (j * L::NCH + c);
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float v = qt[(h0 + h) * kD + d0 + e];
-        qp[(i * 8 + e) * HG + h] = make_float2(fminf(v, 0.f), fmaxf(v, 0.f));
-      }
-  }
-}
-
-// Bounds of `np` (1..8) pages stored at `base` (shared address, 512 B each)
-// for heads [h0, h0 + HG); returns, in the lanes with (lane & 3) == 0, the
-// max over those heads for the task page task_page_of(lane).
-template <int HG>
-__device__ __forceinline__ float bounds_task(uint32_t base, int np, const float2 (&qp)[32], int lane) {
-  using L = BoundsLayout<HG>;
-  const int j = lane % L::LPP, p = lane / L::LPP;
-  const int rot = ((lane & 7) * L::NCH) >> 3;
-  float v[L::NV];
-#pragma unroll
-  for (int s = 0; s < L::STEPS; ++s) {
-    const int tp = s * L::PPS + p;
-    const uint32_t pg = base + static_cast<uint32_t>(tp < np ? tp : 0) * kPageBytes;
-    float2 acc[HG];
-#pragma unroll
-    for (int h = 0; h < HG; ++h) acc[h] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < L::NCH; ++i) {
-      const int c = (i + rot) % L::NCH;
-      const uint32_t off = 16u * static_cast<uint32_t>(j * L::NCH + c);
-      const uint4 lo = lds128(pg + off);
-      const uint4 hi = lds128(pg + 256u + off);
-      const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
-      const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float l = (e & 1) ? bf_hi(wl[e >> 1]) : bf_lo(wl[e >> 1]);
-        const float u = (e & 1) ? bf_hi(wh[e >> 1]) : bf_lo(wh[e >> 1]);
-        const float2 lu = make_float2(l, u);
-#pragma unroll
-        for (int h = 0; h < HG; ++h) acc[h] = __ffma2_rn(lu, qp[(i * 8 + e) * HG + h], acc[h]);
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < HG; ++h) v[s * HG + h] = acc[h].x + acc[h].y;
-  }
-  ReduceScatter<L::NV, L::LPP / 2>::run(v, lane);
-  float u = v[0];
-  if constexpr (HG == 4) {
-    u = fmaxf(u, __shfl_xor_sync(FULL, u, 1));
-    u = fmaxf(u, __shfl_xor_sync(FULL, u, 2));
-  } else if constexpr (HG == 2) {
-    u = fmaxf(u, __shfl_xor_sync(FULL, u, 2));
-  }
-  return u;
-}
-
-// The task page whose bound bounds_task<HG> leaves in `lane`.
-template <int HG>
-__device__ __forceinline__ int task_page_of(int lane) {
-  if constexpr (HG == 4) return 2 * ((lane & 15) >> 2) + (lane >> 4);
-  else if constexpr (HG == 2) return 4 * ((lane >> 2) & 1) + (lane >> 3);
-  else return lane >> 2;
-}
-
-// ------------------------------------------------------------ attention
-
-// Warp-level attention over groups of 8 selected tokens.  Lane l holds dims
-// [4 l, 4 l + 4) of the queries (pre-scaled by scale * log2 e) and of its
-// output accumulators.  Scores: per-lane partial dot products, reduced over
-// the warp by a butterfly; the online softmax is float32 with exp2.
-template <int HA>
-struct AttnLayout {
-  static constexpr int NV = 8 * HA;                       // (token, head) scores per group
-  static constexpr int SHIFT = (NV == 32) ? 0 : (NV == 16) ? 1 : 2;  // lane = idx << SHIFT
-};
-
-template <int RG>
-struct AttnState {
-  static constexpr int HA = RG < 4 ? RG : 4;
-  static constexpr int NPASS = RG / HA;
-  float q[RG][4];
-  float o[RG][4];
-  float m[NPASS], l[NPASS];  // for head (lane >> SHIFT) % HA of each pass
-};
-
-template <int RG>
-__device__ __forceinline__ void attend_group(AttnState<RG>& st, uint32_t kb, uint32_t vb, int nv,
-                                             int lane) {
-  constexpr int HA = AttnState<RG>::HA;
-  constexpr int NV = AttnLayout<HA>::NV;
-  constexpr int SH = AttnLayout<HA>::SHIFT;
-  float kf[8][4];
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const uint2 w = lds64(kb + t * 256u + 8u * lane);
-    kf[t][0] = bf_lo(w.x);
-    kf[t][1] = bf_hi(w.x);
-    kf[t][2] = bf_lo(w.y);
-    kf[t][3] = bf_hi(w.y);
-  }
-  const int t_me = lane >> 2;   // token of this lane's score (NV = 8, 16 or 32)
-#pragma unroll
-  for (int ps = 0; ps < AttnState<RG>::NPASS; ++ps) {
-    float v[NV];
-#pragma unroll
-    for (int t = 0; t < 8; ++t)
-#pragma unroll
-      for (int h = 0; h < HA; ++h) {
-        const float* qh = st.q[ps * HA + h];
-        float2 acc = __fmul2_rn(make_float2(kf[t][0], kf[t][1]), make_float2(qh[0], qh[1]));
-        acc = __ffma2_rn(make_float2(kf[t][2], kf[t][3]), make_float2(qh[2], qh[3]), acc);
-        v[t * HA + h] = acc.x + acc.y;
-      }
-    ReduceScatter<NV, 16>::run(v, lane);
-    const float sc = t_me < nv ? v[0] : -INFINITY;
-    float mx = sc;
-    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
-    const float m_new = fmaxf(st.m[ps], mx);     // finite: the group has a valid token
-    const float alpha = exp2f(st.m[ps] - m_new); // 0 while m is -inf
-    const float p = exp2f(sc - m_new);           // 0 for masked tokens
-    float ps_sum = p;
-    ps_sum += __shfl_xor_sync(FULL, ps_sum, 4);
-    ps_sum += __shfl_xor_sync(FULL, ps_sum, 8);
-    ps_sum += __shfl_xor_sync(FULL, ps_sum, 16);
-    st.l[ps] = fmaf(st.l[ps], alpha, ps_sum);
-    st.m[ps] = m_new;
-#pragma unroll
-    for (int h = 0; h < HA; ++h) {
-      const float ah = __shfl_sync(FULL, alpha, h << SH);   // token 0, head h
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st.o[ps * HA + h][e] *= ah;
-    }
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const uint2 w = lds64(vb + t * 256u + 8u * lane);
-      const float2 v01 = make_float2(bf_lo(w.x), bf_hi(w.x));
-      const float2 v23 = make_float2(bf_lo(w.y), bf_hi(w.y));
-#pragma unroll
-      for (int h = 0; h < HA; ++h) {
-        const float pt = __shfl_sync(FULL, p, (t * HA + h) << SH);
-        float* oh = st.o[ps * HA + h];
-        float2 a01 = __ffma2_rn(v01, make_float2(pt, pt), make_float2(oh[0], oh[1]));
-        float2 a23 = __ffma2_rn(v23, make_float2(pt, pt), make_float2(oh[2], oh[3]));
-        oh[0] = a01.x;
-        oh[1] = a01.y;
-        oh[2] = a23.x;
-        oh[3] = a23.y;
-      }
-    }
-  }
-}
-
-// One warp: the merge weights of n partial softmax states of one head.
-// State i has its running max at st[i * stride + d] and its sum at
-// st[i * stride + d + 1].  Writes wgt[i] = 2^(m_i - M) (M the largest m_i;
-// zero when every state is empty) and hdr = {M, sum_i wgt[i] l_i}.
-template <bool GLOBAL>
-__device__ __forceinline__ float state_ld(const float* p) {
-  if constexpr (GLOBAL) return __ldcg(p);   // written by other CTAs: read at L2
-  else return *p;
-}
-
-template <bool GLOBAL = false>
+// One warp: the merge weights of n partial softmax states of one head (in
+// shared memory).  State i has its running max at st[i * stride + d] and its
+// sum at st[i * stride + d + 1].  Writes wgt[i] = 2^(m_i - M) (M the largest
+// m_i; zero when every state is empty) and hdr = {M, sum_i wgt[i] l_i}.
 __device__ __forceinline__ void merge_weights(const float* st, int stride, int n, float* wgt, float* hdr) {
   const int lane = threadIdx.x & 31;
   float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, state_ld<GLOBAL>(st + i * stride + kD));
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, st[i * stride + kD]);
 #pragma unroll
-  for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
+  for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
   float L = 0.f;
   for (int i = lane; i < n; i += 32) {
-    const float w = (M == -INFINITY) ? 0.f : exp2f(state_ld<GLOBAL>(st + i * stride + kD) - M);
+    const float w = (M == -INFINITY) ? 0.f : exp2f(st[i * stride + kD] - M);
     wgt[i] = w;
-    L = fmaf(state_ld<GLOBAL>(st + i * stride + kD + 1), w, L);
+    L = fmaf(st[i * stride + kD + 1], w, L);
   }
 #pragma unroll
-  for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(FULL, L, o2);
+  for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
   if (lane == 0) {
     hdr[0] = M;
     hdr[1] = L;
   }
 }
 
-// Attention of the group's r heads over `ns` tokens listed in sel[], then the
-// CTA merge of the 16 warp states and the unit merge by the last CTA.
+// ----------------------------------------------------------------------------
+// Phase 6: attention of the r heads over `cnt` tokens listed in sel[], then
+// the per-unit merge.
+//
+// Warp w takes tiles of 16 selected tokens (tiles w, w + 16, ...).  Their K
+// and V rows are staged in the warp's own 8 KB of shared memory (16-B chunk c
+// of token row r at position c ^ (r & 7), so that ldmatrix is conflict-free)
+// and both products run on the tensor cores with fp32 accumulation:
+//   S = Q K^T   m16n8k16, rows = the r heads (bf16 queries, unscaled, so
+//               the products are exact), columns = tokens;
+//   O += P V    rows 0-7 = the bf16 value of each head's softmax weights,
+//               rows 8-15 = the bf16 remainder, so P loses no precision.
+// Online softmax in float32 (exp2 with the scale folded in).  The next
+// tile's K is fetched during the softmax and P V, its V during the next Q K^T.
 template <int RG>
-__device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const int* sel, int ns,
-                                  unsigned char* ring, uint32_t final_target, int* s_int) {
-  using ST = AttnState<RG>;
-  constexpr int HA = ST::HA;
-  constexpr int SH = AttnLayout<HA>::SHIFT;
+__device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const int* sel, int cnt,
+                                  unsigned char* scratch, uint32_t final_target, int* s_int) {
+  static_assert(RG <= 8, "the heads fill at most the upper 8 rows of an m16 tile");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g8 = lane >> 2, t4 = lane & 3;      // mma fragment: row (head), column pair
+  const int lm = lane >> 3, lr = lane & 7;      // ldmatrix: matrix, row
   const int b = unit / a.Hkv, g = unit % a.Hkv;
   const size_t unit_rows = static_cast<size_t>(unit) * a.n_cap;
   const uint16_t* Ku = a.K + unit_rows * kD;
   const uint16_t* Vu = a.V + unit_rows * kD;
 
-  ST st;
-  {
-    const uint16_t* qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * RG) * kD;
-#pragma unroll
-    for (int h = 0; h < RG; ++h) {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(qg + h * kD) + lane);
-      st.q[h][0] = bf_lo(w.x) * a.scale_log2;
-      st.q[h][1] = bf_hi(w.x) * a.scale_log2;
-      st.q[h][2] = bf_lo(w.y) * a.scale_log2;
-      st.q[h][3] = bf_hi(w.y) * a.scale_log2;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st.o[h][e] = 0.f;
-    }
-#pragma unroll
-    for (int ps = 0; ps < ST::NPASS; ++ps) {
-      st.m[ps] = -INFINITY;
-      st.l[ps] = 0.f;
-    }
-  }
-
-  // Per warp two 4-KiB buffers of [K rows 0-7 | V rows 0-7] (256 B each),
-  // filled by cp.async: lane l copies 16-B column chunk l % 16 of rows
-  // l / 16, + 2, ..., one commit group per token group (rows past the end
-  // repeat a valid token, whose softmax weight is zero).
-  unsigned char* wbuf = ring + warp * 8192;
-  const int n_groups = (ns + 7) / 8;
-  auto issue = [&](int gi, int buf) {
-    if (gi < n_groups) {
-      const uint32_t dst = smem_addr(wbuf + buf * 4096);
+  unsigned char* kbuf = scratch + warp * 8192;
+  unsigned char* vbuf = kbuf + 4096;
+  const uint32_t kb_s = smem_addr(kbuf), vb_s = smem_addr(vbuf);
+  const int n_tiles = (cnt + 15) / 16;
+  // every lane: 8 of the tile's 256 16-B chunks of K (or V), one commit group;
+  // rows past cnt are zero-filled
+  auto issue = [&](const uint16_t* base, unsigned char* buf, int tile) {
+    if (tile < n_tiles) {
       const int ch = lane & 15;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int r = (lane >> 4) + 2 * i;            // 0-7: K row, 8-15: V row
-        const int t = r & 7;
-        const int n = sel[min(gi * 8 + t, ns - 1)];
-        const uint16_t* src = (r < 8 ? Ku : Vu) + static_cast<size_t>(n) * kD + ch * 8;
-        cp_async16(dst + r * 256 + ch * 16, src);
+        const int r = (lane >> 4) + 2 * i;
+        const int t = tile * 16 + r;
+        const bool ok = t < cnt;
+        const uint16_t* src = ok ? base + static_cast<size_t>(sel[t]) * kD + ch * 8 : base;
+        cp_async16_zfill(buf + r * 256 + ((ch ^ (r & 7)) << 4), src, ok ? 16u : 0u);
       }
     }
     cp_async_commit();
   };
-  issue(warp, 0);
-  issue(warp + NWARPS, 1);
-  int it = 0;
-  for (int gi = warp; gi < n_groups; gi += NWARPS, ++it) {
-    const int buf = it & 1;
-    cp_async_wait<1>();   // this lane's copies of group gi have landed
+
+  float o[kD / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < kD / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+
+  issue(Ku, kbuf, warp);
+  issue(Vu, vbuf, warp);
+  // The group's queries as the A tile of Q K^T in shared memory (above the
+  // warps' K / V buffers): row h < r is head h, rows r..15 are zero; 16-B
+  // chunk c of row h sits at c ^ (h & 7).  Fragments are read per k-step
+  // with ldmatrix rather than held in registers.
+  unsigned char* qtile = scratch + NWARPS * 8192;
+  if (tid < 16 * 16) {
+    const int h = tid >> 4, ch = tid & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (h < RG) v = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(b) * a.Hq + g * RG + h) * kD) + ch);
+    *reinterpret_cast<uint4*>(qtile + h * 256 + ((ch ^ (h & 7)) << 4)) = v;
+  }
+  __syncthreads();   // (the first K / V tiles are already in flight)
+  const uint32_t q_row = smem_addr(qtile) + ((lm & 1) * 8 + lr) * 256;
+  for (int tile = warp; tile < n_tiles; tile += NWARPS) {
+    cp_async_wait<1>();   // this lane's K chunks of the tile
     __syncwarp();         // ... and every lane's
-    const uint32_t kb = smem_addr(wbuf + buf * 4096);
-    attend_group<RG>(st, kb, kb + 2048, min(8, ns - gi * 8), lane);
-    __syncwarp();         // the buffer has been read
-    issue(gi + 2 * NWARPS, buf);
+    float sacc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll 2
+    for (int ks = 0; ks < kD / 16; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(q_row + (static_cast<uint32_t>((2 * ks + (lm >> 1)) ^ lr) << 4), a0, a1, a2, a3);
+      ldsm_x4(kb_s + ((lm >> 1) * 8 + lr) * 256 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4),
+              b0, b1, b2, b3);
+      mma_bf16_16816(sacc[0], a0, a1, a2, a3, b0, b1);
+      mma_bf16_16816(sacc[1], a0, a1, a2, a3, b2, b3);
+    }
+    __syncwarp();
+    issue(Ku, kbuf, tile + NWARPS);
+
+    // head g8's scores of tokens 2 t4, 2 t4 + 1, 8 + 2 t4, 9 + 2 t4
+    const int valid = cnt - tile * 16;
+    float sc[4] = {sacc[0][0], sacc[0][1], sacc[1][0], sacc[1][1]};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = (e >> 1) * 8 + 2 * t4 + (e & 1);
+      sc[e] = tok < valid ? sc[e] * a.scale_log2 : -INFINITY;
+    }
+    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);       // finite: the tile has a valid token
+    const float alpha = exp2f(m_run - m_new);   // 0 while m_run is -inf
+    float pr[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pr[e] = exp2f(sc[e] - m_new);
+    float ps = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
+    l_run = fmaf(l_run, alpha, ps);
+    m_run = m_new;
+    uint32_t pa[4];
+    {
+      uint16_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat16 h16 = __float2bfloat16_rn(pr[e]);
+        hi[e] = __bfloat16_as_ushort(h16);
+        lo[e] = __bfloat16_as_ushort(__float2bfloat16_rn(pr[e] - __bfloat162float(h16)));
+      }
+      pa[0] = hi[0] | (static_cast<uint32_t>(hi[1]) << 16);   // row g8, tokens 2 t4, + 1
+      pa[1] = lo[0] | (static_cast<uint32_t>(lo[1]) << 16);   // row g8 + 8
+      pa[2] = hi[2] | (static_cast<uint32_t>(hi[3]) << 16);   // row g8, tokens 8 + 2 t4, + 1
+      pa[3] = lo[2] | (static_cast<uint32_t>(lo[3]) << 16);
+    }
+#pragma unroll
+    for (int nt = 0; nt < kD / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][e] *= alpha;
+
+    cp_async_wait<1>();   // this lane's V chunks of the tile
+    __syncwarp();
+#pragma unroll
+    for (int np = 0; np < kD / 16; ++np) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(vb_s + ((lm & 1) * 8 + lr) * 256 + (static_cast<uint32_t>((2 * np + (lm >> 1)) ^ lr) << 4),
+                    b0, b1, b2, b3);
+      mma_bf16_16816(o[2 * np], pa[0], pa[1], pa[2], pa[3], b0, b1);
+      mma_bf16_16816(o[2 * np + 1], pa[0], pa[1], pa[2], pa[3], b2, b3);
+    }
+    __syncwarp();
+    issue(Vu, vbuf, tile + NWARPS);
   }
   cp_async_wait<0>();
-  __syncthreads();        // the merge buffer below overlays the K / V buffers
+  __syncthreads();   // the merge buffer below overlays the K / V tiles
 
-  // merge the 16 warp states through shared memory: [warp][h][MS], the
-  // d outputs then max and sum (rows padded to 16 B)
-  constexpr int MS = kD + 4;
-  float* mer = reinterpret_cast<float*>(ring);
+  // merge the 16 warp states through shared memory: [warp][h][d + 2]
+  float* mer = reinterpret_cast<float*>(scratch);
+  if (g8 < RG) {
+    float* dst = mer + (warp * RG + g8) * (kD + 2);
 #pragma unroll
-  for (int h = 0; h < RG; ++h) {
-    float* dst = mer + (warp * RG + h) * MS;
-    *reinterpret_cast<float4*>(dst + 4 * lane) = make_float4(st.o[h][0], st.o[h][1], st.o[h][2], st.o[h][3]);
+    for (int nt = 0; nt < kD / 8; ++nt) {
+      dst[8 * nt + 2 * t4] = o[nt][0] + o[nt][2];
+      dst[8 * nt + 2 * t4 + 1] = o[nt][1] + o[nt][3];
+    }
+    if (t4 == 0) {
+      dst[kD] = m_run;
+      dst[kD + 1] = l_run;
+    }
   }
-#pragma unroll
-  for (int ps = 0; ps < ST::NPASS; ++ps)
-#pragma unroll
-    for (int h = 0; h < HA; ++h)
-      if (lane == (h << SH)) {
-        float* dst = mer + (warp * RG + ps * HA + h) * MS;
-        dst[kD] = st.m[ps];
-        dst[kD + 1] = st.l[ps];
-      }
   __syncthreads();
 
   constexpr int PS = part_stride(RG);
   float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * PS;
   {
-    float* wgt = mer + NWARPS * RG * MS;         // [RG][NWARPS]
+    // weights e^(m_w - M) of the 16 warp states of each head (warp h does
+    // head h), then thread (h, j) combines the outputs with them
+    float* wgt = mer + NWARPS * RG * (kD + 2);   // [RG][NWARPS]
     float* hdr = wgt + NWARPS * RG;              // [RG][2]: M, sum of weighted l
-    if (warp < RG) merge_weights(mer + warp * MS, RG * MS, NWARPS, wgt + warp * NWARPS, hdr + 2 * warp);
+    if (warp < RG) merge_weights(mer + warp * (kD + 2), RG * (kD + 2), NWARPS, wgt + warp * NWARPS, hdr + 2 * warp);
     __syncthreads();
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
       float O = 0.f;
 #pragma unroll 4
-      for (int w = 0; w < NWARPS; ++w) O = fmaf(mer[(w * RG + h) * MS + j], wgt[h * NWARPS + w], O);
+      for (int w = 0; w < NWARPS; ++w) O = fmaf(mer[(w * RG + h) * (kD + 2) + j], wgt[h * NWARPS + w], O);
       const float L = hdr[2 * h + 1];
       if (a.C == 1) {
         a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
@@ -867,10 +577,9 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   }
 
   // last CTA of the unit merges the C partial states and resets the counter
-  uint32_t* ctr = a.counters + unit;
   __syncthreads();
   if (tid == 0) {
-    const uint32_t old = atom_add_acq_rel(ctr, 1u);
+    const uint32_t old = atom_add_acq_rel(a.counters + unit, 1u);
     s_int[0] = (old == final_target - 1) ? 1 : 0;
     // this CTA's share of the step is done but for the final merge: the
     // next kernel on the stream may start launching (it waits for the
@@ -880,600 +589,572 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   __syncthreads();
   if (!s_int[0]) return;
   if (a.C > 1) {
+    // the C partial states of the unit, copied from L2 in one batch of 16-B
+    // chunks (PS is a multiple of 4 floats); then weights by one warp per
+    // head, and thread (h, j) combines column j of head h
     const float* parts = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit) * PS;
-    float* wgt = mer;                  // [RG][C]
-    float* hdr = wgt + a.C * RG;       // [RG][2]
-    if (warp < RG) merge_weights<true>(parts + warp * (kD + 2), PS, a.C, wgt + warp * a.C, hdr + 2 * warp);
+    float* sp = reinterpret_cast<float*>(scratch);    // [C][PS]
+    float* wgt = sp + a.C * PS;                       // [RG][C]
+    float* hdr = wgt + a.C * RG;                      // [RG][2]
+    for (int i = tid; i < a.C * PS / 4; i += NT) cp_async16(sp + 4 * i, parts + 4 * i);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    if (warp < RG) merge_weights(sp + warp * (kD + 2), PS, a.C, wgt + warp * a.C, hdr + 2 * warp);
     __syncthreads();
     for (int oi = tid; oi < RG * kD; oi += NT) {
       const int h = oi / kD, j = oi % kD;
       float O = 0.f;
 #pragma unroll 6
-      for (int cc = 0; cc < a.C; ++cc) O = fmaf(__ldcg(parts + cc * PS + h * (kD + 2) + j), wgt[h * a.C + cc], O);
+      for (int cc = 0; cc < a.C; ++cc) O = fmaf(sp[cc * PS + h * (kD + 2) + j], wgt[h * a.C + cc], O);
       const float L = hdr[2 * h + 1];
       a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
     }
   }
-  if (tid == 0) atomicExch(ctr, 0u);
-}
-
-// Thread 0 waits until the unit counter reaches `target` (acquire), then the
-// CTA barrier releases everyone.  Returns false (HHR_ERR_TIMEOUT recorded)
-// if the wait ran out.  Every thread of the CTA calls it.
-__device__ bool unit_wait(const uint32_t* ctr, uint32_t target, const DecodeArgs& a, int* s_flag) {
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    const long long t0 = clock64();
-    while (ld_acquire(ctr) < target) {
-      if (static_cast<unsigned long long>(clock64() - t0) > a.spin_limit) {
-        atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-        ok = 0;
-        break;
-      }
-    }
-    *s_flag = ok;
-  }
-  __syncthreads();
-  return *s_flag != 0;
+  if (tid == 0) atomicExch(a.counters + unit, 0u);
 }
 
 // ----------------------------------------------------------------------------
 template <int RG, int WORDS, int MODE>
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int BITS = WORDS * 32;
-  constexpr int HG = RG < 4 ? RG : 4;           // heads per bounds pass
-  constexpr int NPASS = RG / HG;
-  __shared__ __align__(8) unsigned long long s_full[kSlots];
-  __shared__ __align__(8) unsigned long long s_rwbar;
-  __shared__ uint32_t s_slotcnt[kSlots];
-  __shared__ uint32_t s_last[kSlots];           // last chunk (global count) issued into each slot
-  __shared__ int s_scan[NWARPS + 1];
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: wait here, before any global memory access, until that kernel
+  // has completed and its writes are visible.  Only the launch itself
+  // overlaps; no work of two steps does.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int s_int[NWARPS + 16];
   __shared__ int s_scan1[NWARPS];
-  __shared__ int s_misc[32];
-  __shared__ float s_flt[2 * NWARPS];
-  __shared__ int s_cum[kSample + 2];           // own bin counts, then their prefix
-  __shared__ int s_fill[kSample + 1];
-  __shared__ int s_task;                        // next scan task (dynamic assignment)
-  __shared__ int s_cA[kMaxCtasPerUnit], s_cB[kMaxCtasPerUnit], s_cC[kMaxCtasPerUnit], s_cE[kMaxCtasPerUnit];
-  __shared__ int s_dh[BITS + 2];                // distance histogram, then its prefix
-
+  __shared__ int s_aux[264];  // distance totals (<= 257 bins)
+  __shared__ float s_flt[4];
+  constexpr int BITS = WORDS * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x % a.C;
-  const DecodeSmem lay = decode_smem(RG, BITS, a.slice_pages, MODE);
-  unsigned char* ring = smem + lay.ring;
-  float* rw = reinterpret_cast<float*>(smem + lay.rw);
-  float* sS = reinterpret_cast<float*>(smem + lay.sS);
-  uint32_t* sE = reinterpret_cast<uint32_t*>(smem + lay.sE);
-  float* sU = reinterpret_cast<float*>(smem + lay.sU);
-  uint8_t* sBin = smem + lay.sBin;
-  float* qt = reinterpret_cast<float*>(smem + lay.qt);
-  float* qraw = reinterpret_cast<float*>(smem + lay.qraw);
-  uint32_t* qc = reinterpret_cast<uint32_t*>(smem + lay.qc);
-  const uint32_t ring_s = smem_addr(ring);
-  const uint64_t pol_keep = policy_evict_last();
-  const uint32_t rw_bar = smem_addr(&s_rwbar);
+  const DecodeSmem lay = decode_smem(a.NP, a.C, BITS, RG, a.slice_pages, a.slice_tokens, MODE);
+  Smem S;
+  S.qb = reinterpret_cast<uint16_t*>(smem + lay.qb);
+  S.qf = reinterpret_cast<float*>(smem + lay.qf);
+  S.qc = reinterpret_cast<uint32_t*>(smem + lay.qc);
+  S.my_pages = reinterpret_cast<int*>(smem + lay.my_pages);
+  S.tokD = reinterpret_cast<uint16_t*>(smem + lay.tokD);
+  S.sel = reinterpret_cast<int*>(smem + lay.sel);
+  S.scratch = smem + lay.scratch;
+  int* s_scan = s_int;              // NWARPS + 1 entries
+  int* s_misc = s_int + NWARPS + 1; // scalars
+  __shared__ __align__(8) unsigned long long s_rwbar;                       // W staging
+  const uint32_t rw_addr = smem_addr(&s_rwbar);
+  uint32_t rw_seq = 0;  // W phases used so far
   if (tid == 0) {
-    for (int s = 0; s < kSlots; ++s) mbar_init(smem_addr(&s_full[s]), 1u);
-    mbar_init(rw_bar, 1u);
+    mbar_init(rw_addr, 1u);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (tid < kSlots) {
-    s_slotcnt[tid] = 0u;
-    s_last[tid] = 0xFFFFFFFFu;
+  if constexpr (MODE != kModeAttend) {
+    // the B operand's unused columns (fourth term of each head, absent heads) stay zero
+    for (int i = tid; i < 8 * ((RG * 4 + 7) / 8) * 2 * kD; i += NT) S.qb[i] = 0;
   }
-  // Launched as a programmatic dependent of the previous kernel on the
-  // stream: the set-up above touches only shared memory; wait here, before
-  // any global memory access, until that kernel has completed and its
-  // writes are visible.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
-  uint32_t rw_seq = 0;     // phases of the R / W barrier used so far
-  uint32_t chunk0 = 0;     // ring chunks used so far (slot = chunk % kSlots)
 
   for (int unit = blockIdx.x / a.C; unit < a.units; unit += a.grid_units) {
     const int b = unit / a.Hkv, g = unit % a.Hkv;
+
     uint32_t* ctr = a.counters + unit;
 
+    const uint16_t* qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * RG) * kD;
+
     if constexpr (MODE == kModeAttend) {
-      const int n = min(max(a.nsel_in[unit], 0), a.k);
+      const int n = a.nsel_in[unit];
       const int s0 = static_cast<int>(static_cast<long long>(c) * n / a.C);
       const int s1 = static_cast<int>(static_cast<long long>(c + 1) * n / a.C);
-      int* sel = reinterpret_cast<int*>(rw);
       const int32_t* src = a.tok_in + static_cast<size_t>(unit) * a.k;
-      for (int i = s0 + tid; i < s1; i += NT) {
-        const int t = src[i];
-        sel[i - s0] = (t >= 0 && t < a.n_cap) ? t : 0;   // out-of-range indices are clamped
-      }
+#pragma unroll 8
+      for (int i = s0 + tid; i < s1; i += NT) S.sel[i - s0] = src[i];
       __syncthreads();
-      attend_and_finish<RG>(a, unit, c, sel, s1 - s0, ring, static_cast<uint32_t>(a.C), s_misc);
+      attend_and_finish<RG>(a, unit, c, S.sel, s1 - s0, S.scratch, static_cast<uint32_t>(a.C), s_misc);
       __syncthreads();
       continue;
     } else {
-      const int NP = a.NP, Pk = a.Pk, S_ = a.page;
-      const int pb = c * NP / a.C;            // c NP < 2^31: NP <= HHR_MAX_PAGES
-      const int pe = (c + 1) * NP / a.C;
-      const int n_own = pe - pb;
-      const bool local = a.local != 0;
-      const int n_smp = a.n_sample;                      // 0: own pages only (C == 1)
-      const int n_sc = (n_smp + kChunkPages - 1) / kChunkPages;
-      const int n_oc = (local && n_smp > 0) ? 0 : (n_own + kChunkPages - 1) / kChunkPages;
-      const int n_chunks = n_sc + n_oc;
-      const uint16_t* meta_u = a.meta + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
-      const uint16_t* qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * RG) * kD;
+      // ---------------------------------------------------------- phase 0
+      // R reaches shared memory ahead of any metadata.  Every warp streams
+      // its own run of pages into a lane-private ring: the first kLaneSlots
+      // pages of each warp at once, the rest of the ring -- which shares its
+      // storage with R -- as soon as q~ = q R is formed.  W follows by bulk
+      // copy on an mbarrier once the ring has drained.
+      const long long pb = static_cast<long long>(c) * a.NP / a.C;
+      const long long pe = static_cast<long long>(c + 1) * a.NP / a.C;
+      const int my_pages = static_cast<int>(pe - pb);
+      float* sRW = reinterpret_cast<float*>(S.scratch + NWARPS * kLaneSlots * 512);
       const float* Rg = a.R + static_cast<size_t>(g) * kD * kD;
       const float* Wg = a.W + static_cast<size_t>(g) * kD * BITS;
-      // sampled mode: 8 blocks of 8 consecutive pages, block b starting at page b NP / 8
-      auto smp_block = [&](int bl) { return bl * NP / 8; };
-      // chunk k of this unit: the sample's chunks first, then the own pages'
-      auto chunk_pages = [&](int k) {
-        return k < n_sc ? min(kChunkPages, n_smp - k * kChunkPages)
-                        : min(kChunkPages, n_own - (k - n_sc) * kChunkPages);
-      };
-      // one thread: fill ring slot of chunk k (its previous contents are no
-      // longer read by any warp)
-      auto issue_chunk = [&](int k) {
-        const uint32_t gk = chunk0 + static_cast<uint32_t>(k);
-        const uint32_t slot = gk % kSlots;
-        const uint32_t bar = smem_addr(&s_full[slot]);
-        const int np = chunk_pages(k);
-        fence_proxy_async();
-        mbar_expect_tx(bar, static_cast<uint32_t>(np) * kPageBytes);
-        const uint32_t dst = ring_s + slot * kChunkBytes;
-        if (k < n_sc && !local) {
-          for (int bb = 0; bb < kChunkPages / 8; ++bb)
-            bulk_g2s(dst + bb * 8 * kPageBytes, meta_u + static_cast<size_t>(smp_block(k * (kChunkPages / 8) + bb)) * 2 * kD,
-                     8 * kPageBytes, bar);
-        } else {
-          const int p0 = k < n_sc ? k * kChunkPages : pb + (k - n_sc) * kChunkPages;
-          bulk_g2s(dst, meta_u + static_cast<size_t>(p0) * 2 * kD, static_cast<uint32_t>(np) * kPageBytes, bar);
-        }
-        *reinterpret_cast<volatile uint32_t*>(&s_last[slot]) = gk;   // after expect_tx armed the phase
-      };
-
-      // thread 0, after a timed-out wait: record it and wait (bounded) for
-      // every copy this CTA may still have in flight into shared memory
-      auto drain = [&]() {
-        atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-        for (int s2 = 0; s2 < kSlots; ++s2) {
-          const uint32_t last = s_last[s2];
-          if (last != 0xFFFFFFFFu) mbar_wait(smem_addr(&s_full[s2]), (last / kSlots) & 1u, a.spin_limit);
-        }
-        mbar_wait(rw_bar, rw_seq & 1u, a.spin_limit);
-      };
-
-      // ---------------------------------------------------------- phase 0
-      // R by thread 0, which then waits for it; the ring by another warp
-      // (a thread that issues many bulk copies is held back by the copy
-      // engine's queue)
-      if (tid == 0) {
-        fence_proxy_async();
-        mbar_expect_tx(rw_bar, kRWBytes);
-        bulk_g2s_hint(smem_addr(rw), Rg, kRWBytes, rw_bar, pol_keep);
-      }
-      if (tid == 32)
-        for (int k = 0; k < min(kSlots, n_chunks); ++k) issue_chunk(k);
-      for (int i = tid; i < RG * kD; i += NT) qraw[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
-      {
-        const bool okr = (tid == 0) ? mbar_wait(rw_bar, rw_seq & 1u, a.spin_limit) : true;
-        if (__syncthreads_or(!okr)) {
-          if (tid == 0) drain();
-          __syncthreads();
-          return;
-        }
-        ++rw_seq;
-      }
-      if (tid == 0) s_task = NWARPS;     // tasks 0 .. NWARPS-1 go to warps 0 .. NWARPS-1
-      query_product<RG>(qraw, rw, qt);   // q~ = q R (its barriers publish s_task too)
-      if (tid == 0) {                     // W, first 128 columns
-        fence_proxy_async();
-        mbar_expect_tx(rw_bar, kRWBytes);
+      auto issue_w = [&](int half_w) {  // thread 0 only: 128 columns of W
+        // the storage was last touched by generic-proxy copies and loads
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
         if constexpr (BITS == kD) {
-          bulk_g2s_hint(smem_addr(rw), Wg, kRWBytes, rw_bar, pol_keep);
+          bulk_g2s_keep(smem_addr(sRW), Wg, kD * kD * sizeof(float), rw_addr);
         } else {
           for (int i = 0; i < kD; ++i)
-            bulk_g2s_hint(smem_addr(rw + i * kD), Wg + static_cast<size_t>(i) * BITS, kD * 4, rw_bar, pol_keep);
+            bulk_g2s_keep(smem_addr(sRW + i * kD), Wg + static_cast<size_t>(i) * BITS + half_w * kD,
+                     kD * sizeof(float), rw_addr);
         }
-      }
+      };
+      // thread 0 waits for the next W phase; false (all threads) on timeout
+      auto wait_rw = [&]() {
+        const bool ok = (tid == 0) ? mbar_wait(rw_addr, rw_seq & 1u, a.spin_limit) : true;
+        ++rw_seq;
+        return !__syncthreads_or(!ok);
+      };
 
-      // ---------------------------------------------------------- phase 1
-      int err = 0;
-      {
-        float2 qp[32];
-        if constexpr (NPASS == 1) load_qpairs<HG>(qt, 0, qp, lane);
-        const int n_tasks = n_chunks * kTasksPerChunk;
-        // tasks in order, each warp taking the next one when it is free
-        int t = warp;
-        for (; t < n_tasks;) {
-          const int k = t / kTasksPerChunk, jt = t % kTasksPerChunk;
-          const uint32_t gk = chunk0 + static_cast<uint32_t>(k);
-          const uint32_t slot = gk % kSlots;
-          bool got = true;
-          if (lane == 0) {
-            // the slot's barrier phase belongs to chunk gk only once gk has
-            // been issued into it (a parity wait on a later chunk would
-            // otherwise see the previous phase): wait for that first
-            const long long ts = clock64();
-            while (*reinterpret_cast<volatile uint32_t*>(&s_last[slot]) != gk) {
-              if (static_cast<unsigned long long>(clock64() - ts) > a.spin_limit) {
-                got = false;
-                break;
-              }
-            }
-            if (got) got = mbar_wait(smem_addr(&s_full[slot]), (gk / kSlots) & 1u, a.spin_limit);
-          }
-          if (!__shfl_sync(FULL, got ? 1 : 0, 0)) {
-            err = 1;
-            break;
-          }
-          const int np = chunk_pages(k) - jt * kTaskPages;
-          if (np > 0) {
-            const uint32_t base = ring_s + slot * kChunkBytes + jt * kTaskPages * kPageBytes;
-            float u;
-            if constexpr (NPASS == 1) {
-              u = bounds_task<HG>(base, min(np, kTaskPages), qp, lane);
-            } else {
-              load_qpairs<HG>(qt, 0, qp, lane);
-              u = bounds_task<HG>(base, min(np, kTaskPages), qp, lane);
+      // This warp's pages [wpb, wpe).  Lane l only ever reads bytes
+      // [16 l, 16 l + 16) of a page, so it copies exactly those bytes into its
+      // own shared-memory slots with cp.async and waits on its own copies: no
+      // barrier is involved.  Slot s of warp w is the 512 B at
+      // (s * NWARPS + w) * 512: slots [0, kLaneSlots) lie below the R / W
+      // buffer, slots [kLaneSlots, kRingSlots) inside it.
+      const long long wpb = pb + static_cast<long long>(my_pages) * warp / NWARPS;
+      const long long wpe = pb + static_cast<long long>(my_pages) * (warp + 1) / NWARPS;
+      const int w_pages = static_cast<int>(wpe - wpb);
+      constexpr int PPG = 8;                        // pages per ring group; an A tile is two groups
+      constexpr int G0 = 1;                         // groups in flight while q~ is formed (A/B: 1 beats 0 and 2)
+      constexpr int GR = kRingSlots / PPG;          // groups in flight afterwards
+      static_assert(kLaneSlots % PPG == 0 && kRingSlots % PPG == 0 && G0 * PPG <= kLaneSlots,
+                    "whole groups per ring; the groups issued before q~ stay below the R / W buffer");
+      static_assert(GR == 3, "tile ti reads groups 2 ti, 2 ti + 1 and refills them with 2 ti + 3, 2 ti + 4");
+      static_assert((kRingSlots - kLaneSlots) * NWARPS * 512 == kD * kD * sizeof(float),
+                    "the upper ring slots fill the R / W buffer exactly");
+      const int n_grp = (w_pages + PPG - 1) / PPG;
+      const uint16_t* meta_u = a.meta + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
+      const uint4* wsrc = reinterpret_cast<const uint4*>(meta_u + wpb * 2 * kD) + lane;  // 32 x 16 B per page
+      // Within a slot, 16-B chunk c sits at position c ^ (s & 7), so that the
+      // same chunk of 8 consecutive slots covers all banks (ldmatrix below).
+      uint4* ring = reinterpret_cast<uint4*>(S.scratch) + warp * 32;
+      auto issue_group = [&](int gi) {  // every lane: its 16 B of PPG pages, one commit group
+        if (gi < n_grp) {
 #pragma unroll
-              for (int ps = 1; ps < NPASS; ++ps) {
-                load_qpairs<HG>(qt, ps * HG, qp, lane);
-                u = fmaxf(u, bounds_task<HG>(base, min(np, kTaskPages), qp, lane));
-              }
-            }
-            const int tp = task_page_of<HG>(lane);
-            if ((lane & 3) == 0 && tp < np) {
-              const int i = (k < n_sc ? k : k - n_sc) * kChunkPages + jt * kTaskPages + tp;
-              if (k < n_sc) sS[i] = u;
-              else sU[i] = u;
-            }
+          for (int pp = 0; pp < PPG; ++pp) {
+            const int pg = gi * PPG + pp;
+            const int s = pg % kRingSlots;
+            if (pg < w_pages)
+              cp_async16(ring + s * (NWARPS * 32) + (lane ^ (s & 7)), wsrc + static_cast<size_t>(pg) * 32);
           }
-          __syncwarp();
-          int nxt = 0;
-          if (lane == 0) {
-            const uint32_t old = smem_atom_add_acq_rel(&s_slotcnt[slot], 1u);
-            if (old == kTasksPerChunk - 1) {
-              s_slotcnt[slot] = 0u;
-              if (k + kSlots < n_chunks) issue_chunk(k + kSlots);
-            }
-            nxt = atomicAdd(&s_task, 1);
-          }
-          t = __shfl_sync(FULL, nxt, 0);
         }
+        cp_async_commit();
+      };
+
+      // R alone first, one bulk copy: requested together with the metadata
+      // it would land only with the whole first burst
+      if (tid == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
+        bulk_g2s_keep(smem_addr(sRW), Rg, kD * kD * sizeof(float), rw_addr);
       }
-      chunk0 += static_cast<uint32_t>(n_chunks);
-      if (__syncthreads_or(err)) {   // a ring copy never landed
-        if (tid == 0) drain();
+      // queries of the group, as float (raw) -- q~ is derived from these
+      for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
+      if (!wait_rw()) {
+        if (tid == 0) {
+          atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+          mbar_wait(rw_addr, (rw_seq - 1) & 1u, a.spin_limit);   // the copy may still be in flight
+        }
         __syncthreads();
         return;
       }
+#pragma unroll
+      for (int gi = 0; gi < G0; ++gi) issue_group(gi);
+      {
+        float2 acc[RG];
+        product_partials<RG>(S.qf, sRW, acc);
+        __syncthreads();                            // every thread has read R
+        float* part = sRW;                          // [8][r][d] row-group sums, over R
+        store_partials<RG>(acc, part);
+        __syncthreads();
+        for (int oi = tid; oi < RG * kD; oi += NT) {
+          const float qt = product_sum<RG>(part, oi);
+          const int h = oi / kD, j = oi % kD;
+          put_terms(S.qb, 4 * h, j, fminf(qt, 0.f));
+          put_terms(S.qb, 4 * h, kD + j, fmaxf(qt, 0.f));
+        }
+        __syncthreads();
+      }
+      // the upper ring slots now own the R / W storage
+#pragma unroll
+      for (int gi = G0; gi < GR; ++gi) issue_group(gi);
+
+      // ---------------------------------------------------------- phase 1
+      // Eq. 3 as a contraction: with b_h = [min(q~_h, 0) ; max(q~_h, 0)] and a
+      // page's stored bounds [l ; u] (256 bf16), U_p = max_h [l ; u] . b_h.
+      // Each warp multiplies tiles of 16 of its pages -- A fragments loaded
+      // by ldmatrix straight from its ring -- by B = the exact bf16 terms of
+      // the b_h (4 columns per head) on the tensor cores, fp32 accumulation.
+      constexpr int NB = (RG * 4 + 7) / 8;          // n8 column blocks of B
+      float* wsU_u = a.wsU + static_cast<size_t>(unit) * a.np_stride;
+      float lmin = INFINITY, lmax = -INFINITY;
+      const int n_tiles = (w_pages + 15) / 16;
+      const int lm = lane >> 3, lr = lane & 7;      // ldmatrix: matrix, row
+      const int g8 = lane >> 2, t4 = lane & 3;      // mma fragment: row, column pair
+      const uint32_t ring_s = smem_addr(S.scratch) + warp * 512;
+      const uint32_t qb_s = smem_addr(S.qb);
+      for (int ti = 0; ti < n_tiles; ++ti) {
+        cp_async_wait<1>();   // this lane's groups 2 ti and 2 ti + 1 have landed
+        __syncwarp();         // ... and every lane's
+        // A row (lm & 1) * 8 + lr of the tile is page 16 ti + that row
+        const uint32_t a_row = ring_s + (((2 * ti + (lm & 1)) % GR) * PPG + lr) * (NWARPS * 512);
+        float acc[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[nb][e] = 0.f;
+#pragma unroll 4
+        for (int ks = 0; ks < 2 * kD / 16; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a_row + (static_cast<uint32_t>((2 * ks + (lm >> 1)) ^ lr) << 4), a0, a1, a2, a3);
+#pragma unroll
+          for (int nb = 0; nb < NB; nb += 2) {
+            if (nb + 1 < NB) {
+              uint32_t b0, b1, b2, b3;
+              const int n = (nb + (lm >> 1)) * 8 + lr;
+              ldsm_x4(qb_s + n * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1, b2, b3);
+              mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
+              mma_bf16_16816(acc[nb + 1], a0, a1, a2, a3, b2, b3);
+            } else {
+              uint32_t b0, b1;
+              ldsm_x2(qb_s + (nb * 8 + lr) * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1);
+              mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
+            }
+          }
+        }
+        __syncwarp();
+        issue_group(2 * ti + GR);       // refill the slots just read
+        issue_group(2 * ti + GR + 1);
+        // lane (g8, t4) holds columns 8 nb + 2 t4, + 1 (head 2 nb + t4 / 2)
+        // of tile rows g8 and g8 + 8: add the terms, then take the max over
+        // the heads
+        float u0 = -INFINITY, u1 = -INFINITY;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          float s0 = acc[nb][0] + acc[nb][1];
+          float s1 = acc[nb][2] + acc[nb][3];
+          s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
+          s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
+          if (2 * nb + (t4 >> 1) >= RG) {
+            s0 = -INFINITY;
+            s1 = -INFINITY;
+          }
+          u0 = fmaxf(u0, fmaxf(s0, __shfl_xor_sync(0xFFFFFFFFu, s0, 2)));
+          u1 = fmaxf(u1, fmaxf(s1, __shfl_xor_sync(0xFFFFFFFFu, s1, 2)));
+        }
+        if (t4 == 0) {
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const int pl = ti * 16 + g8 + 8 * hr;
+            if (pl < w_pages) {
+              const float u = hr ? u1 : u0;
+              const long long pg = wpb + pl;
+              wsU_u[pg] = u;
+              if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
+              lmin = fminf(lmin, u);
+              lmax = fmaxf(lmax, u);
+            }
+          }
+        }
+      }
+      cp_async_wait<0>();
+      // CTA min / max of its bounds
+#pragma unroll
+      for (int o2 = 16; o2 >= 1; o2 >>= 1) {
+        lmin = fminf(lmin, __shfl_xor_sync(0xFFFFFFFFu, lmin, o2));
+        lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o2));
+      }
+      float* red = reinterpret_cast<float*>(s_aux);
+      if (lane == 0) {
+        red[warp] = lmin;
+        red[NWARPS + warp] = lmax;
+      }
+      // every lane's ring copies have landed and been read: the R / W
+      // storage is free for W
+      __syncthreads();
+      if (warp == 0) {
+        float mn = lane < NWARPS ? red[lane] : INFINITY;
+        float mx = lane < NWARPS ? red[NWARPS + lane] : -INFINITY;
+#pragma unroll
+        for (int o2 = NWARPS / 2; o2 >= 1; o2 >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o2));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o2));
+        }
+        if (lane == 0) {
+          float* mm2 = a.wsMinMax + 2 * static_cast<size_t>(unit * kMaxCtasPerUnit + c);
+          mm2[0] = mn;
+          mm2[1] = mx;
+        }
+      }
+      if (tid == 0) {
+        issue_w(0);
+        // unit barrier 1: arrive now (the release covers the CTA's U through
+        // the CTA barrier above), wait after the query codes
+        atom_add_acq_rel(ctr, 1u);
+      }
+      // query codes (Eq. 10 + sign) from W in shared memory, 128 columns at
+      // a time, while the other CTAs of the unit finish their bounds
+      int w_done = 0;
+      bool q_ok = true;
+      while (w_done < BITS / kD) {
+        q_ok = wait_rw();
+        if (!q_ok) break;
+        float* part = reinterpret_cast<float*>(S.scratch);  // [8][r][d], in the drained ring
+        {
+          float2 acc[RG];
+          product_partials<RG>(S.qf, sRW, acc);
+          store_partials<RG>(acc, part);
+        }
+        __syncthreads();                            // partial sums visible, this W half read
+        if (w_done + 1 < BITS / kD && tid == 0) issue_w(w_done + 1);
+        for (int oi = tid; oi < RG * kD; oi += NT) {  // warp-uniform trip count
+          const float z = product_sum<RG>(part, oi);
+          const uint32_t word = __ballot_sync(0xFFFFFFFFu, z > 0.f);
+          const int h = oi / kD, t = oi % kD;
+          if (lane == 0) S.qc[h * WORDS + w_done * (kD / 32) + t / 32] = word;
+        }
+        ++w_done;
+        if (w_done < BITS / kD) __syncthreads();    // part is rewritten next
+      }
+      if (__syncthreads_or(!q_ok)) {
+        if (tid == 0) {
+          atomicExch(a.status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
+          mbar_wait(rw_addr, (rw_seq - 1) & 1u, a.spin_limit);   // a copy may still be in flight
+        }
+        __syncthreads();
+        return;
+      }
+      if (!unit_wait(ctr, static_cast<uint32_t>(a.C), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 2
-      Pivot pv;
-      pv.all = 0;
-      pv.key = 0u;
-      pv.page = 0;
-      const float* ownU = (local && n_smp > 0) ? sS + pb : sU;
-      if (!local) {
-        // sample order keys, sorted descending (ties by index): the bin edges.
-        // Entry i's rank is counted by NT / kSample threads over slices.
-        static_assert(NT % kSample == 0, "sample ranking splits the comparisons evenly");
-        uint32_t* sK = sE + kSample;   // keys, then ranks (the upper part of sE)
-        int* sR = reinterpret_cast<int*>(sK + kSample);
-        if (tid < kSample) {
-          sK[tid] = order_key(sS[tid]);
-          sR[tid] = 0;
-        }
-        for (int i = tid; i < kSample + 2; i += NT) s_cum[i] = 0;
-        for (int i = tid; i < kSample + 1; i += NT) s_fill[i] = 0;
-        __syncthreads();
-        {
-          constexpr int PARTS = NT / kSample, SL = kSample / PARTS;
-          const int i = tid % kSample, j0 = (tid / kSample) * SL;
-          const uint32_t ki = sK[i];
-          int r = 0;
+      const int NP = a.NP, Pk = a.Pk;
+      float* sU = reinterpret_cast<float*>(S.scratch);
+      int* sHist = reinterpret_cast<int*>(S.scratch + sizeof(float) * align_up(NP, 4));
+      uint32_t* sBits = reinterpret_cast<uint32_t*>(sHist + kBuckets);
+      const int nwords = (NP + 31) / 32;
+      float* sCU = reinterpret_cast<float*>(sBits + align_up(nwords, 4));
+      int* sCP = reinterpret_cast<int*>(sCU + kCandMax);
+      float* sC2U = reinterpret_cast<float*>(sCP + kCandMax);
+      int* sC2P = reinterpret_cast<int*>(sC2U + kCandMax);
+      // all U of the unit, float4 per thread, kept in registers for the
+      // histogram (the tail of a ragged NP goes straight to shared memory)
+      constexpr int kU4 = (HHR_MAX_PAGES / 4 + NT - 1) / NT;
+      const int n4 = NP / 4;
+      float4 ureg[kU4];
+      {
+        const float4* src4 = reinterpret_cast<const float4*>(wsU_u);
 #pragma unroll
-          for (int jj = 0; jj < SL; ++jj) {
-            const uint32_t kj = sK[j0 + jj];
-            r += static_cast<int>(kj > ki) | (static_cast<int>(kj == ki) & static_cast<int>(j0 + jj < i));
-          }
-          atomicAdd(&sR[i], r);
+        for (int u = 0; u < kU4; ++u) {
+          const int i = tid + u * NT;
+          ureg[u] = i < n4 ? __ldcg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        __syncthreads();
-        if (tid < kSample) sE[sR[tid]] = sK[tid];
-        __syncthreads();
-      // own bins: bin(u) = number of edges above u
-        for (int i = tid; i < n_own; i += NT) {
-          const uint32_t ku = order_key(sU[i]);
-          int lo = 0, hi = n_smp;
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (sE[mid] > ku) lo = mid + 1;
-            else hi = mid;
-          }
-          sBin[i] = static_cast<uint8_t>(lo);
-          atomicAdd(&s_cum[lo + 1], 1);
-          if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pb + i] = sU[i];
-        }
-        __syncthreads();
-        if (warp == 0) {   // prefix over the kSample + 2 entries
-          int run = 0;
-          for (int base = 0; base < kSample + 2; base += 32) {
-            int x = base + lane < kSample + 2 ? s_cum[base + lane] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int y = __shfl_up_sync(FULL, x, o);
-              if (lane >= o) x += y;
-            }
-            if (base + lane < kSample + 2) s_cum[base + lane] = run + x;
-            run += __shfl_sync(FULL, x, 31);
-          }
-        }
-        __syncthreads();
-        {
-          // publish: cumulative counts, and the own bounds ordered by bin,
-          // stored centred on the expected cutoff bin
-          int32_t* cum_g = a.wsCum + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * kCumStride;
-          for (int i = tid; i < kSample + 2; i += NT) cum_g[i] = s_cum[i];
-          const int s = a.list_half;
-          int2* list_g = a.wsList + static_cast<size_t>(unit) * a.list_stride + static_cast<size_t>(c) * 2 * s;
-          const int cexp = s_cum[a.b_exp];
-          for (int i = tid; i < n_own; i += NT) {
-            const int bi = sBin[i];
-            const int pos = s_cum[bi] + atomicAdd(&s_fill[bi], 1);
-            list_g[s + pos - cexp] = make_int2(__float_as_int(sU[i]), pb + i);
-          }
-        }
-      } else if (a.dbg_U) {
-        for (int i = tid; i < n_own; i += NT) a.dbg_U[static_cast<size_t>(unit) * a.NP + pb + i] = ownU[i];
+        for (int p = n4 * 4 + tid; p < NP; p += NT) sU[p] = __ldcg(wsU_u + p);
       }
-      // unit barrier 1: arrive (the release covers what this CTA published
-      // through the CTA barrier)
+      for (int i = tid; i < kBuckets; i += NT) sHist[i] = 0;
+      for (int i = tid; i < nwords; i += NT) sBits[i] = 0u;
+      if (warp == 0) {
+        const float* mm2 = a.wsMinMax + 2 * static_cast<size_t>(unit * kMaxCtasPerUnit);
+        float mn = INFINITY, mx = -INFINITY;
+        for (int i = lane; i < a.C; i += 32) {
+          mn = fminf(mn, __ldcg(mm2 + 2 * i));
+          mx = fmaxf(mx, __ldcg(mm2 + 2 * i + 1));
+        }
+#pragma unroll
+        for (int o2 = 16; o2 >= 1; o2 >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o2));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o2));
+        }
+        if (lane == 0) {
+          s_flt[0] = mn;
+          s_flt[1] = mx;
+        }
+      }
+      if (tid == 0) s_misc[2] = 0;
       __syncthreads();
-      if (tid == 0) atom_add_acq_rel(ctr, 1u);
-      if (!local) {
-        // the codes of the pages likely to be kept into L2 (a hint only)
-        const int b_spec = min(a.b_exp + 3, kSample);
+#pragma unroll
+      for (int u = 0; u < kU4; ++u) {
+        const int i = tid + u * NT;
+        if (i < n4) reinterpret_cast<float4*>(sU)[i] = ureg[u];
+      }
+
+      if (Pk >= NP) {
+        for (int p0 = warp * 32; p0 < NP; p0 += NT) {
+          const unsigned word = __ballot_sync(0xFFFFFFFFu, p0 + lane < NP);
+          if (lane == 0) sBits[p0 >> 5] = word;
+        }
+      } else {
+        const float gmin = s_flt[0];
+        const float range = s_flt[1] - gmin;
+        const float inv = (range > 0.f && range <= FLT_MAX) ? static_cast<float>(kBuckets) / range : 0.f;
+        // bin = round((u - gmin) * inv) by one FMA: the 1.5 * 2^23 offset
+        // leaves the rounded integer in the low mantissa bits.  Monotone in u,
+        // and histogram and extraction use the same map, which is all the
+        // selection needs; clamped for any input (NaN included).
+        auto bucket = [&](float u) {
+          const int bk = __float_as_int(fmaf(u - gmin, inv, 12582912.f)) - 0x4B400000;
+          return min(max(bk, 0), kBuckets - 1);
+        };
+#pragma unroll
+        for (int u = 0; u < kU4; ++u) {
+          if (tid + u * NT < n4) {
+            const int b0 = bucket(ureg[u].x), b1 = bucket(ureg[u].y);
+            const int b2 = bucket(ureg[u].z), b3 = bucket(ureg[u].w);
+            atomicAdd(&sHist[b0], 1);
+            atomicAdd(&sHist[b1], 1);
+            atomicAdd(&sHist[b2], 1);
+            atomicAdd(&sHist[b3], 1);
+          }
+        }
+        for (int p = n4 * 4 + tid; p < NP; p += NT) atomicAdd(&sHist[bucket(sU[p])], 1);
+        __syncthreads();
+        find_boundary(sHist, Pk, s_scan, &s_misc[3]);
+        const int bstar = s_misc[3];
+        const int need = Pk - s_misc[4];
+        const int cntB = sHist[bstar];
+        // four bitmap words per warp step (independent chains)
+        if (cntB == need) {
+          for (int p0 = warp * 32; p0 < NP; p0 += 4 * NT) {
+            bool keep[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int p = p0 + u * NT + lane;
+              keep[u] = p < NP && bucket(sU[p]) >= bstar;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int pw = p0 + u * NT;  // warp-uniform
+              const unsigned word = __ballot_sync(0xFFFFFFFFu, keep[u]);
+              if (lane == 0 && pw < NP) sBits[pw >> 5] = word;
+            }
+          }
+        } else if (cntB <= kCandMax) {
+          for (int p0 = warp * 32; p0 < NP; p0 += 4 * NT) {
+            int bk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int p = p0 + u * NT + lane;
+              bk[u] = p < NP ? bucket(sU[p]) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int pw = p0 + u * NT;  // warp-uniform
+              const unsigned word = __ballot_sync(0xFFFFFFFFu, bk[u] > bstar);
+              if (lane == 0 && pw < NP) sBits[pw >> 5] = word;
+              if (bk[u] == bstar) {
+                const int slot = atomicAdd(&s_misc[2], 1);
+                sCU[slot] = sU[pw + lane];
+                sCP[slot] = pw + lane;
+              }
+            }
+          }
+          __syncthreads();
+          int nc = s_misc[2];
+          int need2 = need;
+          const float* fu = sCU;
+          const int* fp = sCP;
+          if (nc > kRankDirect) {
+            // second level: linear bins over the boundary bin's own range
+            float mn = INFINITY, mx = -INFINITY;
+            for (int i = tid; i < nc; i += NT) {
+              mn = fminf(mn, sCU[i]);
+              mx = fmaxf(mx, sCU[i]);
+            }
+#pragma unroll
+            for (int o2 = 16; o2 >= 1; o2 >>= 1) {
+              mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o2));
+              mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o2));
+            }
+            float* red2 = reinterpret_cast<float*>(sC2P + kCandMax);
+            if (lane == 0) {
+              red2[warp] = mn;
+              red2[NWARPS + warp] = mx;
+            }
+            for (int i = tid; i < kBuckets; i += NT) sHist[i] = 0;
+            if (tid == 0) s_misc[2] = 0;
+            __syncthreads();
+            float cmin = INFINITY, cmax = -INFINITY;
+            for (int w2 = 0; w2 < NWARPS; ++w2) {
+              cmin = fminf(cmin, red2[w2]);
+              cmax = fmaxf(cmax, red2[NWARPS + w2]);
+            }
+            const float r2 = cmax - cmin;
+            const float inv2 = (r2 > 0.f && r2 <= FLT_MAX) ? static_cast<float>(kBuckets) / r2 : 0.f;
+            auto bucket2 = [&](float u) {
+              const int bk = __float_as_int(fmaf(u - cmin, inv2, 12582912.f)) - 0x4B400000;
+              return min(max(bk, 0), kBuckets - 1);
+            };
+            for (int i = tid; i < nc; i += NT) atomicAdd(&sHist[bucket2(sCU[i])], 1);
+            __syncthreads();
+            find_boundary(sHist, need, s_scan, &s_misc[5]);
+            const int b2 = s_misc[5];
+            need2 = need - s_misc[6];
+            for (int i = tid; i < nc; i += NT) {
+              const int bk = bucket2(sCU[i]);
+              if (bk > b2) {
+                atomicOr(&sBits[sCP[i] >> 5], 1u << (sCP[i] & 31));
+              } else if (bk == b2) {
+                const int slot = atomicAdd(&s_misc[2], 1);
+                sC2U[slot] = sCU[i];
+                sC2P[slot] = sCP[i];
+              }
+            }
+            __syncthreads();
+            nc = s_misc[2];
+            fu = sC2U;
+            fp = sC2P;
+          }
+          // exact ranking of the remaining boundary pages: larger bound first,
+          // then lower page index
+          for (int i = tid; i < nc; i += NT) {
+            const float u = fu[i];
+            const int pi = fp[i];
+            int rank = 0;
+#pragma unroll 8
+            for (int j = 0; j < nc; ++j) {
+              const float uj = fu[j];
+              rank += (uj > u) || (uj == u && fp[j] < pi);
+            }
+            if (rank < need2) atomicOr(&sBits[pi >> 5], 1u << (pi & 31));
+          }
+        } else {
+          // many equal-looking bounds: exact search for the Pk-th largest key
+          exact_top_pages(sU, NP, Pk, s_scan, sBits);
+        }
+      }
+      __syncthreads();
+      {
+        // the codes of the kept pages of this CTA's own page range into L2:
+        // the compaction below hands them to some CTA's Hamming pass, whose
+        // loads then hit L2 (a hint only; rows clamped to the codes buffer)
         const size_t row_bytes = static_cast<size_t>(WORDS) * 4;
         const char* cbase = reinterpret_cast<const char*>(a.codes + static_cast<size_t>(unit) * a.n_cap * WORDS);
-        for (int i = tid; i < n_own; i += NT) {
-          if (sBin[i] <= b_spec) {
-            const size_t b0 = static_cast<size_t>(pb + i) * S_ * row_bytes;
-            const size_t b1 = min(static_cast<size_t>(pb + i + 1) * S_, static_cast<size_t>(a.n_valid)) * row_bytes;
+        for (long long p = pb + tid; p < pe; p += NT) {
+          if ((sBits[p >> 5] >> (p & 31)) & 1u) {
+            const size_t b0 = static_cast<size_t>(p) * a.page * row_bytes;
+            const size_t b1 = min(static_cast<size_t>(p + 1) * a.page, static_cast<size_t>(a.n_cap)) * row_bytes;
             for (size_t off = b0 & ~static_cast<size_t>(127); off < b1; off += 128) prefetch_l2(cbase + off);
           }
         }
       }
 
-      // query codes (Eq. 10 + sign) from W, 128 columns at a time
-#pragma unroll 1
-      for (int half = 0; half < BITS / kD; ++half) {
-        const bool okw = (tid == 0) ? mbar_wait(rw_bar, rw_seq & 1u, a.spin_limit) : true;
-        if (__syncthreads_or(!okw)) {
-          if (tid == 0) drain();
-          __syncthreads();
-          return;
-        }
-        ++rw_seq;
-        float* partw = reinterpret_cast<float*>(ring);   // [8][r][d]; the ring is free
-        {
-          float2 acc[RG];
-          product_partials<RG>(qraw, rw, acc);
-          store_partials<RG>(acc, partw);
-        }
-        __syncthreads();   // W read by every thread, the partials visible
-        if (half + 1 < BITS / kD && tid == 0) {   // W columns 128-255 into the same buffer
-          fence_proxy_async();
-          mbar_expect_tx(rw_bar, kRWBytes);
-          for (int i = 0; i < kD; ++i)
-            bulk_g2s_hint(smem_addr(rw + i * kD), Wg + static_cast<size_t>(i) * BITS + kD, kD * 4, rw_bar, pol_keep);
-        }
-        for (int oi = tid; oi < RG * kD; oi += NT) {  // warp-uniform trip count
-          const float z = product_sum<RG>(partw, oi);
-          const uint32_t word = __ballot_sync(FULL, z > 0.f);
-          const int h = oi / kD, t = oi % kD;
-          if (lane == 0) qc[h * WORDS + half * (kD / 32) + t / 32] = word;
-        }
-        __syncthreads();
-      }
-
       // ---------------------------------------------------------- phase 3
-      const uint32_t t1 = static_cast<uint32_t>(a.C) + (a.test_extra_stage == 1 ? 1u : 0u);
-      int my_off = 0;   // kept pages of the CTAs before this one
-      if (Pk >= NP) {
-        pv.all = 1;
-        my_off = pb;
-      } else if (local) {
-        const float* allU = n_smp > 0 ? sS : sU;
-        pv = select_pivot(allU, nullptr, 0, NP, Pk, reinterpret_cast<int*>(ring), s_scan, s_misc, s_flt);
-        int cnt = 0;
-        for (int p = tid; p < pb; p += NT) cnt += kept(order_key(allU[p]), p, pv);
-        my_off = block_sum(cnt, s_scan);
-      } else {
-        if (!unit_wait(ctr, t1, a, s_misc)) return;
-        const int C = a.C, s = a.list_half, win = a.win, W2 = 2 * win;
-        constexpr int CS = kSample + 2, CSS = kCumStride;
-        int* gCum = reinterpret_cast<int*>(ring);                                   // [C][CSS]
-        int2* gWin = reinterpret_cast<int2*>(ring + align_up(sizeof(int) * C * CSS, 16));  // [C][2 win]
-        int* gPart = reinterpret_cast<int*>(rw);                                    // [7][CS] (R/W is free)
-        {
-          // one round trip: every CTA's counts, and its list entries
-          // [s - win, s + win) (those inside its area [0, 2 s))
-          copy_rows_async(smem_addr(gCum),
-                          reinterpret_cast<const char*>(a.wsCum + static_cast<size_t>(unit * kMaxCtasPerUnit) * kCumStride),
-                          C, CSS / 4, sizeof(int) * kCumStride, sizeof(int) * CSS, 0, CSS / 4);
-          const int c_lo = max(0, win - s) / 2, c_hi = min(W2, s + win) / 2;   // 16-B chunks = 2 entries
-          copy_rows_async(smem_addr(gWin),
-                          reinterpret_cast<const char*>(a.wsList + static_cast<size_t>(unit) * a.list_stride + (s - win)),
-                          C, win, sizeof(int2) * 2 * s, sizeof(int2) * W2, c_lo, c_hi);
-          cp_async_wait<0>();
-        }
-        __syncthreads();
-        // partial bin totals: thread (part, b) sums rows part, part + 7, ...
-        constexpr int PARTS = NT / CS;
-        if (tid < PARTS * CS) {
-          const int part = tid / CS, bb = tid - part * CS;
-          int x0 = 0, x1 = 0;
-          int cc = part;
-          for (; cc + PARTS < C; cc += 2 * PARTS) {
-            x0 += gCum[cc * CSS + bb];
-            x1 += gCum[(cc + PARTS) * CSS + bb];
-          }
-          if (cc < C) x0 += gCum[cc * CSS + bb];
-          gPart[part * CS + bb] = x0 + x1;
-        }
-        __syncthreads();
-        // warp 0: tot[b] = entries of the unit in bins below b; the boundary
-        // bin b* (tot[b*] < Pk <= tot[b* + 1]); per CTA its entries above b*
-        // (s_cA), in b* (s_cB) and the offset of those among the candidates (s_cC)
-        if (warp == 0) {
-          constexpr int QB = (CS + 31) / 32;
-          int tot[QB];
-#pragma unroll
-          for (int qq = 0; qq < QB; ++qq) {
-            const int bb = lane + 32 * qq;
-            int x = 0;
-            if (bb < CS) {
-#pragma unroll
-              for (int part = 0; part < PARTS; ++part) x += gPart[part * CS + bb];
-            }
-            tot[qq] = x;
-          }
-          // tot is non-decreasing with tot[0] = 0 < Pk: b* = #{b : tot[b] < Pk} - 1
-          int n_lt = 0;
-#pragma unroll
-          for (int qq = 0; qq < QB; ++qq) n_lt += __popc(__ballot_sync(FULL, lane + 32 * qq < CS && tot[qq] < Pk));
-          const int bst = n_lt - 1;
-          int tb = 0, tb1 = 0;
-#pragma unroll
-          for (int qq = 0; qq < QB; ++qq) {
-            const int v = __shfl_sync(FULL, tot[qq], bst & 31);
-            const int v1 = __shfl_sync(FULL, tot[qq], (bst + 1) & 31);
-            if ((bst >> 5) == qq) tb = v;
-            if (((bst + 1) >> 5) == qq) tb1 = v1;
-          }
-          int run = 0, outside = 0;
-          for (int c0 = 0; c0 < C; c0 += 32) {
-            const int cc = c0 + lane;
-            int base = 0, cnt = 0, rel = 0;
-            if (cc < C) {
-              base = gCum[cc * CSS + bst];
-              cnt = gCum[cc * CSS + bst + 1] - base;
-              const int cexp = gCum[cc * CSS + a.b_exp];
-              rel = base - cexp + win;   // first entry within the window row
-              s_cA[cc] = base;
-              s_cB[cc] = cnt;
-              s_cE[cc] = cexp;
-              // the window row holds entries [c_lo, c_hi) chunks: e in [2 c_lo, 2 c_hi)
-              if (cnt > 0 && (rel < 2 * (max(0, win - s) / 2) || rel + cnt > 2 * (min(W2, s + win) / 2))) outside = 1;
-            }
-            int x = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int y = __shfl_up_sync(FULL, x, o);
-              if (lane >= o) x += y;
-            }
-            if (cc < C) s_cC[cc] = run + x - cnt;
-            run += __shfl_sync(FULL, x, 31);
-          }
-          outside = __any_sync(FULL, outside);
-          if (lane == 0) {
-            s_misc[8] = bst;
-            s_misc[5] = Pk - tb;    // need
-            s_misc[6] = tb1 - tb;   // M
-            s_misc[9] = outside;
-          }
-        }
-        __syncthreads();
-        const int need = s_misc[5];
-        const int M = s_misc[6];
-        const bool in_win = s_misc[9] == 0 && M <= (kRWBytes / 8);
-        float* candU;
-        int* candP;
-        int* scratch;
-        if (in_win) {
-          // the boundary bin's entries, from the window rows, into the R/W buffer
-          candU = rw;
-          candP = reinterpret_cast<int*>(rw) + kRWBytes / 8;
-          for (int cc = warp; cc < C; cc += NWARPS) {
-            const int rel = s_cA[cc] - s_cE[cc] + win;
-            for (int o = lane; o < s_cB[cc]; o += 32) {
-              const int2 en = gWin[cc * W2 + rel + o];
-              candU[s_cC[cc] + o] = __int_as_float(en.x);
-              candP[s_cC[cc] + o] = en.y;
-            }
-          }
-          __syncthreads();
-          scratch = reinterpret_cast<int*>(ring);   // the window rows are dead
-        } else {
-          // some CTA's boundary entries lie outside the rows read: read the
-          // boundary bin itself (a second round trip), into the ring
-          candU = reinterpret_cast<float*>(ring);
-          candP = reinterpret_cast<int*>(ring) + kRingBytes / 8;
-          const int2* list_u = a.wsList + static_cast<size_t>(unit) * a.list_stride;
-          for (int cc = 0; cc < C; ++cc) {
-            const int first = s + s_cA[cc] - s_cE[cc];
-            for (int o = tid; o < s_cB[cc]; o += NT) {
-              const int2 en = __ldcg(list_u + static_cast<size_t>(cc) * 2 * s + first + o);
-              candU[s_cC[cc] + o] = __int_as_float(en.x);
-              candP[s_cC[cc] + o] = en.y;
-            }
-          }
-          __syncthreads();
-          scratch = reinterpret_cast<int*>(rw);
-        }
-        pv = select_pivot(candU, candP, 0, M, need, scratch, s_scan, s_misc, s_flt);
-        // kept pages per CTA: all of its entries above the bin plus its
-        // boundary entries that are not below the cutoff
-        for (int cc = warp; cc < C; cc += NWARPS) {
-          int cnt = 0;
-          for (int o = lane; o < s_cB[cc]; o += 32) {
-            const int i = s_cC[cc] + o;
-            cnt += kept(order_key(candU[i]), candP[i], pv);
-          }
-#pragma unroll
-          for (int o2 = 16; o2 >= 1; o2 >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o2);
-          if (lane == 0) s_cA[cc] += cnt;
-        }
-        __syncthreads();
-        if (warp == 0) {
-          int x = 0;
-          for (int cc = lane; cc < c; cc += 32) x += s_cA[cc];
-#pragma unroll
-          for (int o2 = 16; o2 >= 1; o2 >>= 1) x += __shfl_xor_sync(FULL, x, o2);
-          if (lane == 0) s_misc[10] = x;
-        }
-        __syncthreads();
-        my_off = s_misc[10];
-      }
-
-      // own kept pages in ascending order -> my_pages; page_idx
-      int* my_pages = reinterpret_cast<int*>(ring);                       // <= slice_pages
-      uint16_t* tokD = reinterpret_cast<uint16_t*>(ring + align_up(sizeof(int) * a.slice_pages, 16));
-      int nk;
+      const int ks = static_cast<int>(static_cast<long long>(c) * Pk / a.C);
+      const int ke = static_cast<int>(static_cast<long long>(c + 1) * Pk / a.C);
       {
-        // thread t takes own pages [t*span, (t+1)*span)
-        const int span = (n_own + NT - 1) / NT;
-        const int lo = min(n_own, tid * span), hi = min(n_own, lo + span);
+        // thread t owns bitmap words [t*wpt, (t+1)*wpt)
+        const int wpt = (nwords + NT - 1) / NT;
+        const int w0 = tid * wpt, w1 = min(nwords, w0 + wpt);
         int cnt = 0;
-        uint32_t mask = 0u;   // span <= 32 (n_own <= kMaxSlicePages < 32 NT)
-        for (int i = lo; i < hi; ++i) {
-          const bool kp = (local || pv.all) ? kept(order_key(ownU[i]), pb + i, pv)
-                                            : (sBin[i] < s_misc[8] ||
-                                               (sBin[i] == s_misc[8] && kept(order_key(ownU[i]), pb + i, pv)));
-          if (kp) {
-            mask |= 1u << (i - lo);
-            ++cnt;
-          }
-        }
+        for (int wi = w0; wi < w1; ++wi) cnt += __popc(sBits[wi]);
         int tot;
         int pos = block_excl_scan1(cnt, s_scan1, &tot);
-        nk = tot;
         int32_t* pidx = a.page_idx + static_cast<size_t>(unit) * a.P;
-        for (int i = lo; i < hi; ++i) {
-          if ((mask >> (i - lo)) & 1u) {
-            my_pages[pos] = pb + i;
-            if (my_off + pos < a.P) pidx[my_off + pos] = pb + i;
+        for (int wi = w0; wi < w1; ++wi) {
+          uint32_t bits = sBits[wi];
+          while (bits) {
+            const int p = wi * 32 + __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (pos >= ks && pos < ke) S.my_pages[pos - ks] = p;
+            if (c == 0) pidx[pos] = p;
             ++pos;
           }
         }
@@ -1483,146 +1164,135 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       __syncthreads();
 
       // ---------------------------------------------------------- phase 4
-      const int ntok = nk * S_;
-      for (int i = tid; i < BITS + 2; i += NT) s_dh[i] = 0;
-      uint32_t qcr[RG][WORDS];
+      const int S_ = a.page;
+      const int ntok = (ke - ks) * S_;
+      int* sHD = reinterpret_cast<int*>(S.scratch);  // [BITS + 1]
+      for (int i = tid; i <= BITS; i += NT) sHD[i] = 0;
+      uint32_t qc[RG][WORDS];
 #pragma unroll
       for (int h = 0; h < RG; ++h)
 #pragma unroll
-        for (int w = 0; w < WORDS; ++w) qcr[h][w] = qc[h * WORDS + w];
+        for (int w = 0; w < WORDS; ++w) qc[h][w] = S.qc[h * WORDS + w];
       __syncthreads();
-      {
-        const uint32_t* codes_u = a.codes + static_cast<size_t>(unit) * a.n_cap * WORDS;
-        int32_t* dbgD = a.dbg_D ? a.dbg_D + static_cast<size_t>(unit) * a.P * S_ : nullptr;
-        for (int i0 = warp * 32; i0 < ntok; i0 += NT) {
-          const int i = i0 + lane;
-          int D = 0xFFFF;
-          if (i < ntok) {
-            const int slot = i / S_, off = i - slot * S_;
-            const long long n = static_cast<long long>(my_pages[slot]) * S_ + off;
-            if (n < a.n_valid) {
-              uint32_t kc[WORDS];
-              const uint4* cp = reinterpret_cast<const uint4*>(codes_u + n * WORDS);
+      const uint32_t* codes_u = a.codes + static_cast<size_t>(unit) * a.n_cap * WORDS;
+      int32_t* dbgD = a.dbg_D ? a.dbg_D + static_cast<size_t>(unit) * a.P * S_ : nullptr;
+      for (int i0 = warp * 32; i0 < ntok; i0 += NT) {
+        const int i = i0 + lane;
+        int D = 0xFFFF;
+        int slot = 0, off = 0;
+        if (i < ntok) {
+          slot = i / S_;
+          off = i - slot * S_;
+          const long long n = static_cast<long long>(S.my_pages[slot]) * S_ + off;
+          if (n < a.n_valid) {
+            uint32_t kc[WORDS];
+            const uint4* cp = reinterpret_cast<const uint4*>(codes_u + n * WORDS);
 #pragma unroll
-              for (int w4 = 0; w4 < WORDS / 4; ++w4) {
-                const uint4 t = __ldcs(cp + w4);
-                kc[w4 * 4 + 0] = t.x;
-                kc[w4 * 4 + 1] = t.y;
-                kc[w4 * 4 + 2] = t.z;
-                kc[w4 * 4 + 3] = t.w;
-              }
-              int best = 1 << 20;
-#pragma unroll
-              for (int h = 0; h < RG; ++h) {
-                int dist = 0;
-#pragma unroll
-                for (int w = 0; w < WORDS; ++w) dist += __popc(qcr[h][w] ^ kc[w]);
-                best = min(best, dist);
-              }
-              D = best;
+            for (int w4 = 0; w4 < WORDS / 4; ++w4) {
+              const uint4 t = __ldcs(cp + w4);
+              kc[w4 * 4 + 0] = t.x;
+              kc[w4 * 4 + 1] = t.y;
+              kc[w4 * 4 + 2] = t.z;
+              kc[w4 * 4 + 3] = t.w;
             }
-            tokD[i] = static_cast<uint16_t>(D);
-            if (dbgD && my_off + slot < a.P) dbgD[static_cast<size_t>(my_off + slot) * S_ + off] = (D == 0xFFFF) ? -1 : D;
-          }
-          const unsigned grp = __match_any_sync(FULL, D);
-          if (D != 0xFFFF && lane == __ffs(grp) - 1) atomicAdd(&s_dh[D + 1], __popc(grp));
-        }
-        if (c == 0 && dbgD)
-          for (int i = Pk * S_ + tid; i < a.P * S_; i += NT) dbgD[i] = -1;
-      }
-      __syncthreads();
-      // prefix: s_dh[v] = own tokens with D < v, v = 0 .. BITS + 1
-      if (warp == 0) {
-        int run = 0;
-        for (int base = 0; base < BITS + 2; base += 32) {
-          int x = base + lane < BITS + 2 ? s_dh[base + lane] : 0;
+            int best = 1 << 20;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(FULL, x, o);
-            if (lane >= o) x += y;
+            for (int h = 0; h < RG; ++h) {
+              int dist = 0;
+#pragma unroll
+              for (int w = 0; w < WORDS; ++w) dist += __popc(qc[h][w] ^ kc[w]);
+              best = min(best, dist);
+            }
+            D = best;
           }
-          if (base + lane < BITS + 2) s_dh[base + lane] = run + x;
-          run += __shfl_sync(FULL, x, 31);
+          S.tokD[i] = static_cast<uint16_t>(D);
+          if (dbgD) dbgD[static_cast<size_t>(ks + slot) * S_ + off] = (D == 0xFFFF) ? -1 : D;
         }
+        const unsigned grp = __match_any_sync(0xFFFFFFFFu, D);
+        if (D != 0xFFFF && lane == __ffs(grp) - 1) atomicAdd(&sHD[D], __popc(grp));
       }
+      if (c == 0 && dbgD)
+        for (int i = Pk * S_ + tid; i < a.P * S_; i += NT) dbgD[i] = -1;
       __syncthreads();
       {
-        int32_t* row = a.wsCumD + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * a.cumD_stride;
-        for (int i = tid; i < BITS + 2; i += NT) row[i] = s_dh[i];
+        int32_t* hrow = a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * (BITS + 1);
+        for (int i = tid; i <= BITS; i += NT) hrow[i] = sHD[i];
       }
-      // unit barrier 2 (the release by thread 0 covers the CTA's row through
-      // the CTA barrier)
+      // unit barrier 2 (the release by thread 0 covers the CTA's histogram
+      // row through the CTA barrier)
       __syncthreads();
       if (tid == 0) atom_add_acq_rel(ctr, 1u);
-      const uint32_t t2 = 2u * static_cast<uint32_t>(a.C) + (a.test_extra_stage == 2 ? 1u : 0u);
-      if (!unit_wait(ctr, t2, a, s_misc)) return;
+      if (!unit_wait(ctr, 2u * static_cast<uint32_t>(a.C), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 5
-      constexpr int DS = BITS + 2, DSS = (BITS + 2 + 3) / 4 * 4;   // DSS == cumD_stride
-      int* gD = reinterpret_cast<int*>(ring + align_up(sizeof(int) * a.slice_pages, 16) +
-                                       align_up(sizeof(uint16_t) * a.slice_tokens, 16));   // [C][DSS]
-      copy_rows_async(smem_addr(gD),
-                      reinterpret_cast<const char*>(a.wsCumD + static_cast<size_t>(unit * kMaxCtasPerUnit) * DSS),
-                      a.C, DSS / 4, sizeof(int) * DSS, sizeof(int) * DSS, 0, DSS / 4);
-      cp_async_wait<0>();
-      __syncthreads();
-      // partial totals: thread (part, v) sums rows part, part + PD, ...
-      constexpr int PD = NT / DS;
-      int* dPart = reinterpret_cast<int*>(rw);   // [PD][DS] (R/W is free)
-      if (tid < PD * DS) {
-        const int part = tid / DS, v = tid - part * DS;
-        int x0 = 0, x1 = 0;
-        int cc = part;
-        for (; cc + PD < a.C; cc += 2 * PD) {
-          x0 += gD[cc * DSS + v];
-          x1 += gD[(cc + PD) * DSS + v];
-        }
-        if (cc < a.C) x0 += gD[cc * DSS + v];
-        dPart[part * DS + v] = x0 + x1;
+      int* sHA = reinterpret_cast<int*>(S.scratch);  // [C][BITS + 1]
+      {
+        // one batch of 16-B copies (a plain load/store loop would wait out an
+        // L2 round trip per element, the compiler cannot reorder the global
+        // loads past the shared stores).  The unit's area holds
+        // kMaxCtasPerUnit rows of a multiple of 16 B, so rounding the copy up
+        // to whole chunks stays inside it.
+        const char* hall = reinterpret_cast<const char*>(a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit) * (BITS + 1));
+        const int chunks = (a.C * (BITS + 1) * 4 + 15) / 16;
+        for (int i = tid; i < chunks; i += NT) cp_async16(reinterpret_cast<char*>(sHA) + 16 * i, hall + 16 * i);
+        cp_async_commit();
+        cp_async_wait<0>();
       }
       __syncthreads();
-      // warp 0: tot[v] = tokens of the unit with distance < v; k_eff; the
-      // threshold T (tot[T] < k_eff <= tot[T + 1]); then, in CTA order, each
-      // CTA's quota of ties at T and its output offset
-      if (warp == 0) {
-        constexpr int QV = (DS + 31) / 32;
-        int tot[QV];
-#pragma unroll
-        for (int qq = 0; qq < QV; ++qq) {
-          const int v = lane + 32 * qq;
-          int x = 0;
-          if (v < DS) {
-#pragma unroll
-            for (int part = 0; part < PD; ++part) x += dPart[part * DS + v];
-          }
-          tot[qq] = x;
+      // distance totals tot[v] = sum over the CTAs (thread v); one block-wide
+      // exclusive scan of them gives k_eff, the threshold distance T (the
+      // k_eff-th smallest) and how many tokens at T are still needed
+      int* sbe = sHA + a.C * (BITS + 1);                 // [C][2]: below T, at T
+      if (tid == 0) {
+        s_misc[4] = 0;
+        s_misc[5] = -1;
+      }
+      {
+        int x = 0;
+        if (tid <= BITS) {
+#pragma unroll 6
+          for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * (BITS + 1) + tid];
         }
-        const int total = __shfl_sync(FULL, tot[(DS - 1) / 32], (DS - 1) % 32);
+        int total;
+        const int excl = block_excl_scan(x, s_scan, &total);
         const int k_eff = min(a.k, total);
-        int n_lt = 0;
-#pragma unroll
-        for (int qq = 0; qq < QV; ++qq) n_lt += __popc(__ballot_sync(FULL, lane + 32 * qq < DS && tot[qq] < k_eff));
-        const int T = k_eff > 0 ? n_lt - 1 : -1;   // tot[0] = 0 < k_eff
-        int tT = 0;
-#pragma unroll
-        for (int qq = 0; qq < QV; ++qq) {
-          const int v = __shfl_sync(FULL, tot[qq], T & 31);
-          if (T >= 0 && (T >> 5) == qq) tT = v;
+        if (x > 0 && excl < k_eff && excl + x >= k_eff) {   // exactly one thread
+          s_misc[5] = tid;
+          s_misc[4] = k_eff - excl;
         }
-        if (lane == 0) {
-          s_misc[11] = T;
-          s_misc[15] = k_eff;
+        if (tid == 0) s_misc[6] = k_eff;
+      }
+      __syncthreads();
+      {
+        // per-CTA tokens below T / at T: a half-warp per CTA row
+        const int T = s_misc[5];
+        // warp-uniform trip count: each warp takes rows base and base + 1
+        for (int base = warp * 2; base < a.C; base += NT / 16) {
+          const int cc = base + (lane >> 4), part = lane & 15;
+          const bool row_ok = cc < a.C;
+          int below = 0;
+          if (row_ok)
+            for (int v = part; v < T; v += 16) below += sHA[cc * (BITS + 1) + v];
+#pragma unroll
+          for (int o2 = 8; o2 >= 1; o2 >>= 1) below += __shfl_xor_sync(0xFFFFFFFFu, below, o2);
+          if (row_ok && part == 0) {
+            sbe[2 * cc] = below;
+            sbe[2 * cc + 1] = T >= 0 ? sHA[cc * (BITS + 1) + T] : 0;
+          }
         }
-        const int needT = T >= 0 ? k_eff - tT : 0;
+      }
+      __syncthreads();
+      if (warp == 0) {  // in CTA order: tie quota and output offset of each CTA
+        const int needT = s_misc[4];
         int pre_eq = 0, off = 0;
         for (int c0 = 0; c0 < a.C; c0 += 32) {
           const int cc = c0 + lane;
-          const int below = (cc < a.C && T >= 0) ? gD[cc * DSS + T] : 0;
-          const int eq = (cc < a.C && T >= 0) ? gD[cc * DSS + T + 1] - below : 0;
+          const int below = cc < a.C ? sbe[2 * cc] : 0;
+          const int eq = cc < a.C ? sbe[2 * cc + 1] : 0;
           int eq_in = eq;
 #pragma unroll
           for (int o2 = 1; o2 < 32; o2 <<= 1) {
-            const int y = __shfl_up_sync(FULL, eq_in, o2);
+            const int y = __shfl_up_sync(0xFFFFFFFFu, eq_in, o2);
             if (lane >= o2) eq_in += y;
           }
           const int quota = max(0, min(needT - (pre_eq + eq_in - eq), eq));
@@ -1630,29 +1300,28 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           int sel_in = selc;
 #pragma unroll
           for (int o2 = 1; o2 < 32; o2 <<= 1) {
-            const int y = __shfl_up_sync(FULL, sel_in, o2);
+            const int y = __shfl_up_sync(0xFFFFFFFFu, sel_in, o2);
             if (lane >= o2) sel_in += y;
           }
           if (cc == c) {
-            s_misc[12] = off + sel_in - selc;
-            s_misc[13] = quota;
-            s_misc[14] = selc;
+            s_misc[7] = off + sel_in - selc;
+            s_misc[8] = quota;
+            s_misc[9] = selc;
           }
-          pre_eq += __shfl_sync(FULL, eq_in, 31);
-          off += __shfl_sync(FULL, sel_in, 31);
+          pre_eq += __shfl_sync(0xFFFFFFFFu, eq_in, 31);
+          off += __shfl_sync(0xFFFFFFFFu, sel_in, 31);
         }
       }
       __syncthreads();
-      const int T = s_misc[11], k_eff = s_misc[15];   // threshold distance (-1: nothing selected)
-      const int tok_off = s_misc[12], my_quota = s_misc[13], my_sel = s_misc[14];
-      int* sel = reinterpret_cast<int*>(rw);   // this CTA's selected tokens (ascending)
+      const int T = s_misc[5], k_eff = s_misc[6];
+      const int my_off = s_misc[7], my_quota = s_misc[8], my_sel = s_misc[9];
       {
         // one packed scan: (tokens below T) | (tokens at T) << 16
         const int span = (ntok + NT - 1) / NT;
-        const int lo = min(ntok, tid * span), hi = min(ntok, lo + span);
+        const int lo = tid * span, hi = min(ntok, lo + span);
         int lt = 0, eq = 0;
         for (int i = lo; i < hi; ++i) {
-          const int D = tokD[i];
+          const int D = S.tokD[i];
           lt += D < T;
           eq += D == T;
         }
@@ -1661,7 +1330,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         int lt_b = pre & 0xFFFF, eq_b = pre >> 16;
         int32_t* tout = a.tok_idx + static_cast<size_t>(unit) * a.k;
         for (int i = lo; i < hi; ++i) {
-          const int D = tokD[i];
+          const int D = S.tokD[i];
           int pos = -1;
           if (D < T) {
             pos = lt_b + min(eq_b, my_quota);
@@ -1672,9 +1341,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           }
           if (pos >= 0) {
             const int slot = i / S_;
-            const int n = my_pages[slot] * S_ + (i - slot * S_);
-            if (tok_off + pos < a.k) tout[tok_off + pos] = n;
-            sel[pos] = n;
+            const int n = S.my_pages[slot] * S_ + (i - slot * S_);
+            tout[my_off + pos] = n;
+            S.sel[pos] = n;
           }
         }
         if (c == 0) {
@@ -1685,8 +1354,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       __syncthreads();
 
       if constexpr (MODE == kModeFused) {
-        const uint32_t t3 = 3u * static_cast<uint32_t>(a.C);
-        attend_and_finish<RG>(a, unit, c, sel, my_sel, ring, t3, s_misc);
+        attend_and_finish<RG>(a, unit, c, S.sel, my_sel, S.scratch, 3u * static_cast<uint32_t>(a.C), s_misc);
       } else {
         if (tid == 0) {
           const uint32_t old = atom_add_acq_rel(ctr, 1u);

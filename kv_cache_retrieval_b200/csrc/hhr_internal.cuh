@@ -11,21 +11,16 @@
 
 namespace hhr {
 
-constexpr int kD = 128;                  // head dimension handled by every kernel
-constexpr int kDecodeThreads = 512;      // one decode CTA per SM, 16 warps
-constexpr int kMaxCtasPerUnit = 64;      // CTAs that may share one (sequence, KV head)
-constexpr int kMinPagesPerCta = 32;      // below this a unit uses fewer CTAs
-constexpr int kPageBytes = 2 * kD * 2;   // one page's bf16 [lower; upper] rows
-constexpr int kChunkPages = 32;          // pages per bulk copy of the metadata ring
-constexpr int kChunkBytes = kChunkPages * kPageBytes;  // 16 KiB
-constexpr int kSlots = 8;                // metadata ring slots (128 KiB)
-constexpr int kRingBytes = kSlots * kChunkBytes;
-constexpr int kRWBytes = kD * kD * 4;    // R, or 128 columns of W, in float32
-constexpr int kSample = 64;              // pages every CTA of a unit scores to fix common bins
-constexpr int kLocalMaxPages = 256;      // at most this many pages: every CTA scores all of them
-constexpr int kMaxSlicePages = 2560;     // pages one CTA scores
-constexpr int kMaxTokensPerCta = 8192;   // candidate tokens one CTA ranks
-constexpr int kWinMax = 512;             // list entries read around the expected cutoff, per side
+constexpr int kD = 128;                 // head dimension handled by every kernel
+constexpr int kDecodeThreads = 512;     // one decode CTA per SM, 16 warps
+constexpr int kMaxCtasPerUnit = 64;     // CTAs that may share one (sequence, KV head)
+constexpr int kMinPagesPerCta = 32;     // below this a unit uses fewer CTAs
+constexpr int kBuckets = 2048;          // page top-P histogram bins
+constexpr int kCandMax = 1024;          // boundary-bucket candidates held in shared memory
+constexpr int kRankDirect = 48;         // at most this many are ranked without a second level
+constexpr int kMaxTokensPerCta = 16384; // candidate tokens one CTA scores
+constexpr int kLaneSlots = 16;         // ring slots per warp below the R / W buffer (8 KiB)
+constexpr int kRingSlots = 24;         // ring slots per warp in all (12 KiB), the upper 8 over R / W
 constexpr unsigned long long kSpinLimit = 1ull << 31;  // ~1 s at 2 GHz
 
 inline __host__ __device__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -34,16 +29,10 @@ inline __host__ __device__ size_t align_up(size_t x, size_t a) { return (x + a -
 // padded to a multiple of four so it can be moved with 16-B accesses.
 inline __host__ __device__ constexpr int part_stride(int r) { return (r * (kD + 2) + 3) / 4 * 4; }
 
-// Entries of the cumulative bin counts one CTA publishes for the page
-// selection (kSample + 1 bins -> kSample + 2 prefix values), padded.
-constexpr int kCumStride = (kSample + 2 + 3) / 4 * 4;
-
-// Workspace layout (bytes).  The status word sits at offset 0, the per-unit
-// barrier counters right after it.
+// Workspace layout (bytes).  The status word sits at offset 0.
 struct WsLayout {
-  size_t status, counters, cum, list, cumD, part, total;
-  int list_stride;   // list entries (8 B) per unit
-  int cumD_stride;   // int32 per (unit, CTA) in the distance area
+  size_t status, counters, U, minmax, hist, part, total;
+  int np_stride;  // floats per unit in the U area (multiple of 4)
 };
 
 inline __host__ __device__ WsLayout ws_layout(int units, int np_cap, int r, int bits) {
@@ -51,13 +40,10 @@ inline __host__ __device__ WsLayout ws_layout(int units, int np_cap, int r, int 
   size_t off = 0;
   L.status = off;   off += 256;
   L.counters = off; off += align_up(sizeof(uint32_t) * (size_t)units, 256);
-  L.cum = off;      off += align_up(sizeof(int32_t) * (size_t)units * kMaxCtasPerUnit * kCumStride, 256);
-  // every CTA's list lives in [2 c s, 2 (c + 1) s) with s = ceil(NP / C) rounded up to even,
-  // so 2 C s <= 2 (np_cap + 2 C)
-  L.list_stride = (int)align_up(2 * ((size_t)np_cap + 2 * kMaxCtasPerUnit), 4);
-  L.list = off;     off += align_up(8 * (size_t)units * L.list_stride, 256);
-  L.cumD_stride = (int)align_up((size_t)bits + 2, 4);
-  L.cumD = off;     off += align_up(sizeof(int32_t) * (size_t)units * kMaxCtasPerUnit * L.cumD_stride, 256);
+  L.np_stride = (int)align_up((size_t)np_cap, 4);
+  L.U = off;        off += align_up(sizeof(float) * (size_t)units * L.np_stride, 256);
+  L.minmax = off;   off += align_up(sizeof(float) * 2 * (size_t)units * kMaxCtasPerUnit, 256);
+  L.hist = off;     off += align_up(sizeof(int32_t) * (size_t)units * kMaxCtasPerUnit * (bits + 1), 256);
   L.part = off;     off += align_up(sizeof(float) * (size_t)units * kMaxCtasPerUnit * part_stride(r), 256);
   L.total = off;
   return L;
@@ -86,23 +72,17 @@ struct DecodeArgs {
   // workspace
   uint32_t* status;
   uint32_t* counters;
-  int32_t* wsCum;           // [units][kMaxCtasPerUnit][kCumStride]
-  int2* wsList;             // [units][list_stride] (float bits of U, page)
-  int32_t* wsCumD;          // [units][kMaxCtasPerUnit][cumD_stride]
-  float* wsPart;            // [units][kMaxCtasPerUnit][part_stride]
-  int list_stride, cumD_stride;
+  float* wsU;
+  float* wsMinMax;
+  int32_t* wsHist;
+  float* wsPart;
+  int np_stride;
   // sizes
   int B, Hq, Hkv, units, page, n_cap, np_cap, n_valid, NP, P, Pk, k, C, grid_units;
-  int slice_pages;          // max pages one CTA scores (ceil(NP / C)), 0 in attend mode
-  int slice_tokens;         // max tokens one CTA ranks or attends
-  int local;                // 1: every CTA holds every bound (no page exchange)
-  int n_sample;             // pages of the common sample (NP in local mode when C > 1)
-  int b_exp;                // bin where the page cutoff is expected
-  int win;                  // list entries read on each side of the expected cutoff (even)
-  int list_half;            // half of each CTA's list area (slice_pages rounded up to even)
+  int slice_pages;          // max kept pages one CTA scores (ceil(Pk / C))
+  int slice_tokens;         // max tokens one CTA scores or attends
   float scale_log2;         // scale * log2(e)
   unsigned long long spin_limit;
-  int test_extra_stage;     // test hook: unit barrier (1..3) that waits for one extra arrival, 0 = none
 };
 
 struct EncodeArgs {
@@ -112,32 +92,49 @@ struct EncodeArgs {
   uint32_t* codes;
   uint16_t* meta;
   int Hkv, units, bits, page, n_cap, np_cap, n_begin, n_end, tile_begin, n_tiles;
-  unsigned long long spin_limit;
-  int test_short_tx;        // test hook: expect 16 more bytes than a key tile delivers
 };
 
-// Shared-memory carve-up of a decode CTA (host and device agree on it).
+// Shared-memory bytes of a decode CTA (host and device agree on the carve-up).
 struct DecodeSmem {
-  size_t ring, rw, sS, sE, sU, sBin, qt, qraw, qc, total;
+  size_t qb, qf, qc, my_pages, tokD, sel, scratch, total;
 };
 
-inline __host__ __device__ DecodeSmem decode_smem(int r, int bits, int slice_pages, int mode) {
+inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, int r, int mode) {
+  size_t sel = 0, hist = 0, attn = 0, stream = 0;
+  if (mode != kModeAttend) {
+    // per-warp metadata rings; their upper slots double as R / W staging
+    stream = (size_t)(kDecodeThreads / 32) * kRingSlots * 512;
+    sel = sizeof(float) * align_up((size_t)NP, 4)          // U of every page
+        + sizeof(int) * kBuckets                             // histogram
+        + sizeof(uint32_t) * align_up(((size_t)NP + 31) / 32, 4)  // kept bitmap
+        + 2 * (sizeof(float) + sizeof(int)) * kCandMax       // boundary candidates, 2 levels
+        + sizeof(float) * 2 * (kDecodeThreads / 32);          // level-2 min / max
+    hist = sizeof(int) * ((size_t)C * (bits + 1) + 2 * (size_t)C) + 16;
+  }
+  if (mode != kModeSelect) {
+    // per warp: K and V of 16 tokens; then the 16-row query tile
+    const size_t ring = (size_t)(kDecodeThreads / 32) * 2 * 16 * 2 * kD + 16 * 2 * kD;
+    size_t merge = sizeof(float) * ((kDecodeThreads / 32) * (size_t)r * (kD + 2) + (kDecodeThreads / 32) * (size_t)r + 2 * (size_t)r);
+    const size_t parts = sizeof(float) * ((size_t)C * part_stride(r) + (size_t)C * r + 2 * (size_t)r);  // final merge
+    merge = merge > parts ? merge : parts;
+    attn = ring > merge ? ring : merge;
+  }
+  size_t m = sel > hist ? sel : hist;
+  m = m > stream ? m : stream;
+  return m > attn ? m : attn;
+}
+
+inline __host__ __device__ DecodeSmem decode_smem(int NP, int C, int bits, int r, int slice_pages,
+                                                  int slice_tokens, int mode) {
   DecodeSmem s;
   size_t off = 0;
-  s.ring = off;  off += kRingBytes;                 // metadata ring; later K/V tiles, lists, merges
-  s.rw = off;    off += kRWBytes;                   // R, then W; later the selected tokens
-  if (mode == kModeAttend) {
-    s.sS = s.sE = s.sU = s.sBin = s.qt = s.qraw = s.qc = off;
-    s.total = off;
-    return s;
-  }
-  s.sS = off;    off += sizeof(float) * kLocalMaxPages;            // sample bounds (all, in local mode)
-  s.sE = off;    off += sizeof(float) * kLocalMaxPages;            // sorted sample (bin edges)
-  s.sU = off;    off += align_up(sizeof(float) * (size_t)slice_pages, 16);   // own bounds
-  s.sBin = off;  off += align_up((size_t)slice_pages, 16);                  // own bins (u8)
-  s.qt = off;    off += align_up(sizeof(float) * (size_t)r * kD, 16);      // q~ (float32)
-  s.qraw = off;  off += align_up(sizeof(float) * (size_t)r * kD, 16);      // q (float32)
-  s.qc = off;    off += align_up(sizeof(uint32_t) * (size_t)r * (bits / 32), 16);
+  s.qb = off;       off += (size_t)8 * ((r * 4 + 7) / 8) * 2 * kD * 2;  // bf16 terms of q~, [8 nb][2 d]
+  s.qf = off;       off += align_up(sizeof(float) * r * kD, 16);
+  s.qc = off;       off += align_up(sizeof(uint32_t) * r * (bits / 32), 16);
+  s.my_pages = off; off += align_up(sizeof(int) * (size_t)(slice_pages + 1), 16);
+  s.tokD = off;     off += align_up(sizeof(uint16_t) * (size_t)(slice_tokens + 1), 16);
+  s.sel = off;      off += align_up(sizeof(int) * (size_t)(slice_tokens + 1), 16);
+  s.scratch = off;  off += align_up(decode_scratch_bytes(NP, C, bits, r, mode), 16);
   s.total = off;
   return s;
 }

@@ -56,7 +56,7 @@ extern "C" int32_t hhr_decode_step_noalloc(const hhr_dims* dims, const void* q, 
       hhr::ws_layout(dims->B * dims->Hkv, (dims->n_cap + dims->page - 1) / dims->page,
                      dims->Hq / dims->Hkv, dims->bits);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, L.cum, s) != cudaSuccess) return HHR_ERR_CUDA;
+  if (cudaMemsetAsync(scratch, 0, L.U, s) != cudaSuccess) return HHR_ERR_CUDA;
   return hhr_decode_step(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page_idx, tok_idx,
                          n_sel, out, scratch, HHR_NOALLOC_SCRATCH_BYTES, stream);
 }
