@@ -403,6 +403,7 @@ __device__ __forceinline__ void merge_weights(const float* st, int stride, int n
 // tile's K is fetched during the softmax and P V, its V during the next Q K^T.
 template <int RG>
 __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const int* sel, int cnt,
+                                  const float* qf,
                                   unsigned char* scratch, uint32_t final_target, int* s_int) {
   static_assert(RG <= 8, "the heads fill at most the upper 8 rows of an m16 tile");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -451,7 +452,18 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   if (tid < 16 * 16) {
     const int h = tid >> 4, ch = tid & 15;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (h < RG) v = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(b) * a.Hq + g * RG + h) * kD) + ch);
+    if (h < RG) {
+      if (qf) {   // the group's queries are already in shared memory as float (exact bf16 values)
+        const float4 lo = *reinterpret_cast<const float4*>(qf + h * kD + ch * 8);
+        const float4 hi = *reinterpret_cast<const float4*>(qf + h * kD + ch * 8 + 4);
+        v.x = (__float_as_uint(lo.x) >> 16) | (__float_as_uint(lo.y) & 0xFFFF0000u);
+        v.y = (__float_as_uint(lo.z) >> 16) | (__float_as_uint(lo.w) & 0xFFFF0000u);
+        v.z = (__float_as_uint(hi.x) >> 16) | (__float_as_uint(hi.y) & 0xFFFF0000u);
+        v.w = (__float_as_uint(hi.z) >> 16) | (__float_as_uint(hi.w) & 0xFFFF0000u);
+      } else {
+        v = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(b) * a.Hq + g * RG + h) * kD) + ch);
+      }
+    }
     *reinterpret_cast<uint4*>(qtile + h * 256 + ((ch ^ (h & 7)) << 4)) = v;
   }
   __syncthreads();   // (the first K / V tiles are already in flight)
@@ -669,7 +681,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
 #pragma unroll 8
       for (int i = s0 + tid; i < s1; i += NT) S.sel[i - s0] = src[i];
       __syncthreads();
-      attend_and_finish<RG>(a, unit, c, S.sel, s1 - s0, S.scratch, static_cast<uint32_t>(a.C), s_misc);
+      attend_and_finish<RG>(a, unit, c, S.sel, s1 - s0, nullptr, S.scratch, static_cast<uint32_t>(a.C), s_misc);
       __syncthreads();
       continue;
     } else {
@@ -1354,7 +1366,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       __syncthreads();
 
       if constexpr (MODE == kModeFused) {
-        attend_and_finish<RG>(a, unit, c, S.sel, my_sel, S.scratch, 3u * static_cast<uint32_t>(a.C), s_misc);
+        attend_and_finish<RG>(a, unit, c, S.sel, my_sel, S.qf, S.scratch, 3u * static_cast<uint32_t>(a.C), s_misc);
       } else {
         if (tid == 0) {
           const uint32_t old = atom_add_acq_rel(ctr, 1u);
