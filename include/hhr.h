@@ -243,14 +243,26 @@ int32_t hhr_decode_step_noalloc(const hhr_dims* dims, const void* q, const float
 int32_t hhr_read_status(void* workspace, void* stream);
 
 /*
- * Test hook for the bounded-wait path: launches one CTA that waits on a
- * workspace counter that nothing increments, giving up after `spin_cycles`
- * clock cycles (capped at 2^32).  The expected status afterwards, through
- * hhr_read_status, is HHR_ERR_TIMEOUT.  Needs at least 4096 bytes of zeroed
- * workspace.
+ * Test hook for the bounded waits of the real kernels.  No counterpart in the
+ * paper: it exercises the kernels' failure path without any fault.  Arms a
+ * one-shot, process-wide flag consumed by the next matching call:
+ *   where = 1: the next hhr_select / hhr_decode_step waits at its first unit
+ *              barrier (after the page bounds) for one CTA arrival more than
+ *              the unit has;
+ *   where = 2: the same at its second unit barrier (after the Hamming
+ *              distances);
+ *   where = 3: the next hhr_encode_keys gives its first pipeline stage one
+ *              producer arrival too many, so no tile ever reaches the tensor
+ *              cores.
+ * That call's waits give up after `spin_cycles` clock cycles (clamped to
+ * [1000, 2^32]) instead of about a second, record HHR_ERR_TIMEOUT (read it with
+ * hhr_read_status for 1 and 2, hhr_encode_status for 3) and return; nothing
+ * is left in flight.  After a decode timeout the workspace must be
+ * zero-filled again before the next call.  Outputs of the failed call are
+ * unspecified.  Returns HHR_ERR_INVALID_ARG for another `where`.  Not for
+ * concurrent use.
  */
-int32_t hhr_test_wait_timeout(void* workspace, size_t ws_bytes, uint64_t spin_cycles,
-                              void* stream);
+int32_t hhr_test_arm_timeout(int32_t where, uint64_t spin_cycles);
 
 #ifdef __cplusplus
 }

@@ -61,7 +61,7 @@ _SIGS = {
                                        _I32, C.c_float, _P, _P, _P, _P, _P]),
     "hhr_read_status": (_I32, [_P, _P]),
     "hhr_encode_status": (_I32, [_P]),
-    "hhr_test_wait_timeout": (_I32, [_P, C.c_size_t, C.c_uint64, _P]),
+    "hhr_test_arm_timeout": (_I32, [_I32, C.c_uint64]),
 }
 
 
@@ -183,7 +183,6 @@ def hhr_encode_status(stream=None) -> int:
     return st
 
 
-def hhr_test_wait_timeout(workspace, spin_cycles, ws_bytes=None, stream=None) -> None:
-    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
-    _check(lib().hhr_test_wait_timeout(_ptr(workspace), ws_bytes, spin_cycles, _stream(stream)),
-           "hhr_test_wait_timeout")
+def hhr_test_arm_timeout(where, spin_cycles) -> None:
+    """Test hook: the next matching call's bounded waits run out (see hhr.h)."""
+    _check(lib().hhr_test_arm_timeout(where, spin_cycles), "hhr_test_arm_timeout")

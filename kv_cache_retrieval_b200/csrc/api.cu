@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -157,6 +158,20 @@ int32_t check_workspace(const hhr_dims* d, void* ws, size_t ws_bytes) {
 
 int32_t finish_launch(cudaError_t e) { return e == cudaSuccess ? HHR_OK : HHR_ERR_CUDA; }
 
+// One-shot test hook (hhr_test_arm_timeout): which wait the next matching
+// call makes unmeetable, and the spin limit it gets.
+std::atomic<int> g_test_where{0};
+std::atomic<unsigned long long> g_test_spin{0};
+
+// Consumes the hook when it is armed for one of the given sites.
+int take_test_hook(int lo, int hi, unsigned long long* spin) {
+  int w = g_test_where.load();
+  if (w < lo || w > hi) return 0;
+  if (!g_test_where.compare_exchange_strong(w, 0)) return 0;
+  *spin = g_test_spin.load();
+  return w;
+}
+
 }  // namespace
 
 
@@ -198,6 +213,15 @@ int32_t hhr_encode_keys(const hhr_dims* dims, const void* K, const float* R, con
   a.np_cap = np_cap_of(dims);
   a.n_begin = n_begin;
   a.n_end = n_end;
+  a.spin_limit = kSpinLimit;
+  a.test_extra_arrival = 0;
+  {
+    unsigned long long spin = 0;
+    if (take_test_hook(3, 3, &spin)) {
+      a.test_extra_arrival = 1;
+      a.spin_limit = spin;
+    }
+  }
   a.tile_begin = n_begin / kEncodeTileKeys * kEncodeTileKeys;
   a.n_tiles = (n_end - a.tile_begin + kEncodeTileKeys - 1) / kEncodeTileKeys;
   DeviceInfo info;
@@ -255,6 +279,13 @@ static int32_t decode_common(const hhr_dims* dims, int mode, const void* q, cons
   a.dbg_U = dbg_U;
   a.dbg_D = dbg_D;
   a.scale_log2 = scale * 1.4426950408889634f;
+  if (mode != kModeAttend) {
+    unsigned long long spin = 0;
+    if (const int w = take_test_hook(1, 2, &spin)) {
+      a.test_extra_stage = w;
+      a.spin_limit = spin;
+    }
+  }
   carve_workspace(workspace, dims, &a);
   return finish_launch(launch_decode(a, dims->Hq / dims->Hkv, dims->bits, mode, smem,
                                      static_cast<cudaStream_t>(stream)));
@@ -307,14 +338,13 @@ int32_t hhr_read_status(void* workspace, void* stream) {
   return static_cast<int32_t>(host);
 }
 
-int32_t hhr_test_wait_timeout(void* workspace, size_t ws_bytes, uint64_t spin_cycles, void* stream) {
-  if (!workspace || ws_bytes < 4096 || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return HHR_ERR_WORKSPACE;
+int32_t hhr_test_arm_timeout(int32_t where, uint64_t spin_cycles) {
+  if (where < 1 || where > 3) return HHR_ERR_INVALID_ARG;
+  if (spin_cycles < 1000) spin_cycles = 1000;
   if (spin_cycles > (1ull << 32)) spin_cycles = 1ull << 32;
-  unsigned char* base = static_cast<unsigned char*>(workspace);
-  uint32_t* status = reinterpret_cast<uint32_t*>(base);
-  uint32_t* counter = reinterpret_cast<uint32_t*>(base + 256);
-  return finish_launch(launch_wait_timeout(status, counter, spin_cycles, static_cast<cudaStream_t>(stream)));
+  g_test_spin.store(spin_cycles);
+  g_test_where.store(where);
+  return HHR_OK;
 }
 
 }  // extern "C"

@@ -935,7 +935,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         __syncthreads();
         return;
       }
-      if (!unit_wait(ctr, static_cast<uint32_t>(a.C), a, s_misc)) return;
+      if (!unit_wait(ctr, static_cast<uint32_t>(a.C) + (a.test_extra_stage == 1 ? 1u : 0u), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 2
       const int NP = a.NP, Pk = a.Pk;
@@ -1234,7 +1234,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // row through the CTA barrier)
       __syncthreads();
       if (tid == 0) atom_add_acq_rel(ctr, 1u);
-      if (!unit_wait(ctr, 2u * static_cast<uint32_t>(a.C), a, s_misc)) return;
+      if (!unit_wait(ctr, 2u * static_cast<uint32_t>(a.C) + (a.test_extra_stage == 2 ? 1u : 0u), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 5
       int* sHA = reinterpret_cast<int*>(S.scratch);  // [C][BITS + 1]
@@ -1379,18 +1379,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
   }
 }
 
-__global__ void wait_timeout_kernel(uint32_t* status, uint32_t* counter, unsigned long long spin) {
-  if (threadIdx.x != 0) return;
-  const long long t0 = clock64();
-  while (ld_acquire(counter) < 1u) {
-    if (static_cast<unsigned long long>(clock64() - t0) > spin) {
-      atomicExch(status, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
-      return;
-    }
-    __nanosleep(64);
-  }
-}
-
 template <int RG, int WORDS, int MODE>
 cudaError_t launch_t(const DecodeArgs& a, size_t smem, cudaStream_t stream) {
   auto kern = decode_kernel<RG, WORDS, MODE>;
@@ -1445,12 +1433,6 @@ cudaError_t launch_decode(const DecodeArgs& a, int r, int bits, int mode, size_t
     case 8: return launch_bits<8>(a, bits, mode, smem_bytes, stream);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_wait_timeout(uint32_t* status, uint32_t* counter, unsigned long long spin,
-                                cudaStream_t stream) {
-  wait_timeout_kernel<<<1, 32, 0, stream>>>(status, counter, spin);
-  return cudaGetLastError();
 }
 
 }  // namespace hhr

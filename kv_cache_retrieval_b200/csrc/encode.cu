@@ -39,7 +39,6 @@ constexpr int kMmaWarp = kEpiWarps + kProdWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kAccCols = 128;                        // fp32 TMEM columns per accumulator
 constexpr uint32_t kTmemCols = 2 * kAccCols;              // double-buffered
-constexpr unsigned long long kWaitLimit = 1ull << 31;     // clock cycles, about one second
 // kind::f16 instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
@@ -76,13 +75,13 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 // Waits for the completion of the phase with the given parity; false (and the
-// sticky error set) once kWaitLimit cycles have passed.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// sticky error set) once `limit` cycles have passed.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long limit) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   do {
     if (mbar_try(bar, parity)) return true;
-  } while (static_cast<unsigned long long>(clock64() - t0) <= kWaitLimit);
+  } while (static_cast<unsigned long long>(clock64() - t0) <= limit);
   atomicExch(&g_encode_err, static_cast<uint32_t>(HHR_ERR_TIMEOUT));
   return false;
 }
@@ -252,7 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a)
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&bar_full[s]), kProdWarps * 32);
+      // (the test hook makes the first stage wait for one arrival more than
+      // the producers make: every role's wait then runs out and the kernel
+      // leaves through its normal exit, with no MMA issued)
+      mbar_init(smem_u32(&bar_full[s]), kProdWarps * 32 + (a.test_extra_arrival && s == 0 ? 1 : 0));
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a)
     int lq = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++lq) {
       const int s = lq % kStages;
-      if (!mbar_wait(smem_u32(&bar_empty[s]), ((lq / kStages) & 1) ^ 1)) break;
+      if (!mbar_wait(smem_u32(&bar_empty[s]), ((lq / kStages) & 1) ^ 1, a.spin_limit)) break;
       const int unit = (it / a.n_tiles) * a.Hkv + g;
       const int key0 = a.tile_begin + (it % a.n_tiles) * kTileKeys;
       const uint16_t* Ku = a.K + static_cast<size_t>(unit) * a.n_cap * kD;
@@ -308,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a)
       bool ok = true;
       for (int it = blockIdx.x; it < items && ok; it += gridDim.x, ++lq) {
         const int s = lq % kStages, acc = lq & 1;
-        ok = mbar_wait(smem_u32(&bar_acc_empty[acc]), ((lq >> 1) & 1) ^ 1);
-        if (ok) ok = mbar_wait(smem_u32(&bar_full[s]), (lq / kStages) & 1);
+        ok = mbar_wait(smem_u32(&bar_acc_empty[acc]), ((lq >> 1) & 1) ^ 1, a.spin_limit);
+        if (ok) ok = mbar_wait(smem_u32(&bar_full[s]), (lq / kStages) & 1, a.spin_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * kAccCols;
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a)
         tc_commit(smem_u32(&bar_acc_full[acc]));
       }
       // every issued MMA has completed before TMEM is released
-      if (lq > 0) mbar_wait(smem_u32(&bar_acc_full[(lq - 1) & 1]), ((lq - 1) >> 1) & 1);
+      if (lq > 0) mbar_wait(smem_u32(&bar_acc_full[(lq - 1) & 1]), ((lq - 1) >> 1) & 1, a.spin_limit);
     }
     __syncwarp();
   } else {
@@ -336,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a)
     int lq = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++lq) {
       const int acc = lq & 1;
-      if (!mbar_wait(smem_u32(&bar_acc_full[acc]), (lq >> 1) & 1)) break;
+      if (!mbar_wait(smem_u32(&bar_acc_full[acc]), (lq >> 1) & 1, a.spin_limit)) break;
       tc_fence_after();
       const int unit = (it / a.n_tiles) * a.Hkv + g;
       const int key0 = a.tile_begin + (it % a.n_tiles) * kTileKeys;

@@ -83,6 +83,7 @@ struct DecodeArgs {
   int slice_tokens;         // max tokens one CTA scores or attends
   float scale_log2;         // scale * log2(e)
   unsigned long long spin_limit;
+  int test_extra_stage;     // test hook: unit barrier (1 or 2) that waits for one arrival too many; 0 = none
 };
 
 struct EncodeArgs {
@@ -92,6 +93,8 @@ struct EncodeArgs {
   uint32_t* codes;
   uint16_t* meta;
   int Hkv, units, bits, page, n_cap, np_cap, n_begin, n_end, tile_begin, n_tiles;
+  unsigned long long spin_limit;   // clock cycles a pipeline wait may take
+  int test_extra_arrival;          // test hook: the first stage waits for one producer arrival too many
 };
 
 // Shared-memory bytes of a decode CTA (host and device agree on the carve-up).
@@ -166,7 +169,5 @@ size_t encode_smem_bytes();
 // Copies the encode kernels' sticky error word to *out and clears it (synchronizes `stream`).
 cudaError_t encode_read_status(uint32_t* out, cudaStream_t stream);
 constexpr int kEncodeTileKeys = 128;   // keys per encode tile (tile starts are multiples of it)
-cudaError_t launch_wait_timeout(uint32_t* status, uint32_t* counter, unsigned long long spin,
-                                cudaStream_t stream);
 
 }  // namespace hhr
