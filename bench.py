@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the secondary workload lines")
+    ap.add_argument("--workload-steps", type=int, default=3000)
     return ap.parse_args()
 
 
@@ -244,12 +246,166 @@ def aggregate(us_step_max: float, world: int, keys_per_step: int) -> dict:
 
 # ----------------------------------------------------------------- our arm
 
+NOMINAL_HBM_GBS = 8000.0   # the HBM figure the roofline target is stated against
+
+
+class Layers:
+    """Device state of one workload for the timed loop: `n` independent layer
+    instances (their own K, V, codes, metadata, R, W, query and outputs), so
+    that a cycle over them touches more than L2, and one workspace."""
+
+    def __init__(self, w, inp, n, dev):
+        import numpy as np
+        import torch
+        import kv_cache_retrieval_b200 as hhr
+
+        def bf(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+        self.w, self.dev = w, dev
+        self.dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap)
+        K0, V0 = bf(inp.K), bf(inp.V)
+        R0, W0 = torch.from_numpy(inp.R).to(dev), torch.from_numpy(inp.W).to(dev)
+        self.q_all = bf(inp.q)                       # [steps][B][Hq][d]
+        codes0 = torch.zeros(w.B, w.Hkv, w.n_cap, w.words, dtype=torch.int32, device=dev)
+        meta0 = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=torch.bfloat16, device=dev)
+        hhr.hhr_encode_keys(self.dims, K0, R0, W0, 0, w.N, codes0, meta0)
+        self.lay = []
+        for li in range(n):
+            first = li == 0
+            self.lay.append(dict(
+                K=K0 if first else K0.clone(), V=V0 if first else V0.clone(),
+                R=R0 if first else R0.clone(), W=W0 if first else W0.clone(),
+                codes=codes0 if first else codes0.clone(), meta=meta0 if first else meta0.clone(),
+                q=self.q_all[0].clone(),
+                page_idx=torch.empty(w.B, w.Hkv, w.P, dtype=torch.int32, device=dev),
+                tok_idx=torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=dev),
+                n_sel=torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev),
+                out=torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)))
+        self.ws = torch.zeros(hhr.hhr_workspace_size(self.dims, w.P, w.k), dtype=torch.uint8, device=dev)
+        self.scale = 1.0 / math.sqrt(w.d)
+
+    def step(self, li, stream=None, n_valid=None, q=None):
+        import kv_cache_retrieval_b200 as hhr
+        L, w = self.lay[li], self.w
+        hhr.hhr_decode_step(self.dims, L["q"] if q is None else q, L["R"], L["W"], L["codes"], L["meta"],
+                            L["K"], L["V"], w.N if n_valid is None else n_valid, w.P, w.k, self.scale,
+                            L["page_idx"], L["tok_idx"], L["n_sel"], L["out"], self.ws, None, stream)
+
+    def append(self, li, i, stream=None):
+        """Encode the key at position N + i (one decode step's append)."""
+        import kv_cache_retrieval_b200 as hhr
+        L, w = self.lay[li], self.w
+        hhr.hhr_encode_keys(self.dims, L["K"], L["R"], L["W"], w.N + i, w.N + i + 1, L["codes"], L["meta"],
+                            stream)
+
+
+def graph_time_us(body, n_body_steps, total_steps, warmup):
+    """Device time per step of `total_steps` steps: `body(stream)` enqueues
+    n_body_steps steps and is captured once in a CUDA graph, replayed
+    total_steps / n_body_steps times between CUDA events on the replay
+    stream (eager launches if capture fails)."""
+    import torch
+    for _ in range(max(3, warmup)):
+        body(None)
+    torch.cuda.synchronize()
+    reps = max(1, total_steps // n_body_steps)
+    launch = "cuda-graph"
+    g = None
+    try:
+        cs = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs, capture_error_mode="relaxed"):
+            body(cs.cuda_stream)
+        g.replay()
+        torch.cuda.synchronize()
+    except Exception as exc:  # noqa: BLE001
+        launch = f"stream (graph capture failed: {type(exc).__name__})"
+        g = None
+        torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        if g is not None:
+            g.replay()
+        else:
+            body(None)
+    e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1000.0 / (reps * n_body_steps), reps * n_body_steps, launch
+
+
+def encode_ms(lay, w, reps=5):
+    import torch
+    import kv_cache_retrieval_b200 as hhr
+    L = lay.lay[0]
+    s = torch.cuda.current_stream()
+    for _ in range(2):
+        hhr.hhr_encode_keys(lay.dims, L["K"], L["R"], L["W"], 0, w.N, L["codes"], L["meta"])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        hhr.hhr_encode_keys(lay.dims, L["K"], L["R"], L["W"], 0, w.N, L["codes"], L["meta"])
+    e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def workload_line(name, steps, warmup, dev, peak):
+    """One secondary workload: device µs per step (its appends inside the
+    timed steps when it has any), the roofline fraction of its algorithmic
+    bytes, its key encoding and the planted-key recall."""
+    import torch
+    import kv_cache_retrieval_b200 as hhr
+    from workloads import get, make_inputs
+    w = get(name)
+    inp = make_inputs(w)
+    per_step = algorithmic_bytes(w, w.N, w.P, w.k)[1]
+    n_layers = max(1, min(12, int(math.ceil(2.2 * 126e6 / max(per_step, 1)))))   # > 2x L2 per cycle
+    lay = Layers(w, inp, n_layers, dev)
+    enc = encode_ms(lay, w)
+    if w.appends:
+        # one step = append the next key, then decode with it (the graph
+        # re-encodes the same keys on every replay: the merge is idempotent)
+        def body(stream):
+            for i in range(w.appends):
+                lay.append(0, i, stream)
+                lay.step(0, stream, n_valid=w.N + i + 1, q=lay.q_all[i])
+        us, n, launch = graph_time_us(body, w.appends, steps, warmup)
+        per_step = algorithmic_bytes(w, w.N + w.appends, w.P, w.k)[1]
+    else:
+        def body(stream):
+            for li in range(n_layers):
+                lay.step(li, stream)
+        us, n, launch = graph_time_us(body, n_layers, steps, warmup)
+    st = hhr.hhr_read_status(lay.ws)
+    L0 = lay.lay[0]
+    try:
+        recall = planted_recall(L0["tok_idx"].cpu().numpy(), L0["n_sel"].cpu().numpy(),
+                                L0["page_idx"].cpu().numpy(), inp.planted_pos, w.page)
+    except Exception as exc:  # noqa: BLE001
+        recall = {"error": f"{type(exc).__name__}: {exc}"}
+    achieved = per_step / (us * 1e-6) / 1e9
+    out = {"us_per_step": round(us, 3), "steps": n, "layers_cycled": n_layers, "launch": launch,
+           "appends_in_step": bool(w.appends), "algorithmic_bytes": per_step,
+           "achieved_gbs": round(achieved, 1), "frac": round(achieved / peak, 4),
+           "frac_vs_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+           "keys_scored_per_s": w.B * w.Hkv * w.N / (us * 1e-6),
+           "encode_ms": round(enc, 4), "planted_recall": recall, "status": hhr.hhr_status_string(st)}
+    del lay, inp
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_hhr(args):
     import numpy as np
     import torch
     import torch.distributed as dist
 
     import kv_cache_retrieval_b200 as hhr
+    from kv_cache_retrieval_b200 import _binding as Bnd
     from kv_cache_retrieval_b200 import build as kbuild
     from workloads import get, make_inputs
 
@@ -272,58 +428,20 @@ def run_hhr(args):
     inp = make_inputs(w)
     n_valid = w.N
     L = max(1, args.layers)
-    dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap)
-
-    def bf(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
-
-    K0, V0 = bf(inp.K), bf(inp.V)
-    q_host = torch.from_numpy(np.ascontiguousarray(inp.q[0]).view(np.int16)).view(torch.bfloat16)
-    q_dev = q_host.to(dev)
-    R = torch.from_numpy(inp.R).to(dev)
-    W = torch.from_numpy(inp.W).to(dev)
-    codes0 = torch.zeros(w.B, w.Hkv, w.n_cap, w.words, dtype=torch.int32, device=dev)
-    meta0 = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=torch.bfloat16, device=dev)
-
-    # key encoding of the whole context, timed separately
-    s = torch.cuda.current_stream()
-    for _ in range(2):
-        hhr.hhr_encode_keys(dims, K0, R, W, 0, n_valid, codes0, meta0)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 5
-    e0.record(s)
-    for _ in range(reps):
-        hhr.hhr_encode_keys(dims, K0, R, W, 0, n_valid, codes0, meta0)
-    e1.record(s)
-    torch.cuda.synchronize()
-    enc_ms = e0.elapsed_time(e1) / reps
+    lay = Layers(w, inp, L, dev)
+    dims = lay.dims
+    enc_ms = encode_ms(lay, w)
     enc_flops = 2.0 * w.B * w.Hkv * n_valid * w.d * (w.d + w.bits)
 
-    layers = []
-    for li in range(L):
-        lay = dict(
-            K=K0 if li == 0 else K0.clone(), V=V0 if li == 0 else V0.clone(),
-            codes=codes0 if li == 0 else codes0.clone(), meta=meta0 if li == 0 else meta0.clone(),
-            q=q_dev.clone(), R=R if li == 0 else R.clone(), W=W if li == 0 else W.clone(),
-            page_idx=torch.empty(w.B, w.Hkv, w.P, dtype=torch.int32, device=dev),
-            tok_idx=torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=dev),
-            n_sel=torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev),
-            out=torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev))
-        layers.append(lay)
-    ws = torch.zeros(hhr.hhr_workspace_size(dims, w.P, w.k), dtype=torch.uint8, device=dev)
-    scale = 1.0 / math.sqrt(w.d)
-
-    def step(lay, stream=None):
-        hhr.hhr_decode_step(dims, lay["q"], lay["R"], lay["W"], lay["codes"], lay["meta"], lay["K"], lay["V"],
-                            n_valid, w.P, w.k, scale, lay["page_idx"], lay["tok_idx"], lay["n_sel"],
-                            lay["out"], ws, None, stream)
+    def body(stream):
+        for li in range(L):
+            lay.step(li, stream)
 
     # warm-up (eager), then one CUDA graph per cycle over the layer instances
     for i in range(max(3, args.warmup)):
-        step(layers[i % L])
+        lay.step(i % L)
     torch.cuda.synchronize()
-    assert hhr.hhr_read_status(ws) == hhr.HHR_OK
+    assert hhr.hhr_read_status(lay.ws) == hhr.HHR_OK
 
     K = max(1, args.steps)
     launch = "cuda-graph"
@@ -334,7 +452,7 @@ def run_hhr(args):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="relaxed"):
                 for li in range(n):
-                    step(layers[li], cap_stream.cuda_stream)
+                    lay.step(li, cap_stream.cuda_stream)
             graphs[n] = g
         for g in graphs.values():
             g.replay()
@@ -361,7 +479,7 @@ def run_hhr(args):
             graphs[K % L].replay()
     else:
         for i in range(K):
-            step(layers[i % L])
+            lay.step(i % L)
     ev1.record(s)
     torch.cuda.synchronize()
     t1 = time.time()
@@ -371,7 +489,7 @@ def run_hhr(args):
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
-    status = hhr.hhr_read_status(ws)
+    status = hhr.hhr_read_status(lay.ws)
     assert status == hhr.HHR_OK, hhr.hhr_status_string(status)
 
     us_step = ms * 1000.0 / K
@@ -383,28 +501,30 @@ def run_hhr(args):
     peak, peak_kind = measured_peak()
     achieved = alg / (us_step * 1e-6) / 1e9
 
-    # end to end through the public API: pinned q in, decode, out back
-    q_pin = q_host.pin_memory()
+    # end to end through the public API: one blocking call per step that
+    # copies the pinned host query in, decodes and copies the output back
+    q_pin = torch.from_numpy(np.ascontiguousarray(inp.q[0]).view(np.int16)).view(torch.bfloat16).pin_memory()
     out_pin = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32).pin_memory()
-    lay0 = layers[0]
+    calls = []
+    for li in range(L):
+        Lr = lay.lay[li]
+        calls.append(Bnd.prepare("hhr_decode_step_host", dims, q_pin, Lr["q"], Lr["R"], Lr["W"], Lr["codes"],
+                                 Lr["meta"], Lr["K"], Lr["V"], n_valid, w.P, w.k, lay.scale, Lr["page_idx"],
+                                 Lr["tok_idx"], Lr["n_sel"], Lr["out"], out_pin, lay.ws,
+                                 lay.ws.numel(), torch.cuda.current_stream().cuda_stream))
     n_e2e = max(1, min(args.e2e_steps, K))
-    for _ in range(20):
-        lay0["q"].copy_(q_pin, non_blocking=True)
-        step(lay0)
-        out_pin.copy_(lay0["out"], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+    for i in range(20):
+        calls[i % L]()
     if world > 1:
         dist.barrier()
     te0 = time.perf_counter()
     for i in range(n_e2e):
-        lay = layers[i % L]
-        lay["q"].copy_(q_pin, non_blocking=True)
-        step(lay)
-        out_pin.copy_(lay["out"], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+        calls[i % L]()
     te1 = time.perf_counter()
     e2e_us = max_over_ranks((te1 - te0) * 1e6 / n_e2e, dev)
+    assert hhr.hhr_read_status(lay.ws) == hhr.HHR_OK
 
+    lay0 = lay.lay[0]
     try:   # a diagnostic: it must not cost the bench line
         recall = planted_recall(lay0["tok_idx"].cpu().numpy(), lay0["n_sel"].cpu().numpy(),
                                 lay0["page_idx"].cpu().numpy(), inp.planted_pos, w.page)
@@ -414,6 +534,20 @@ def run_hhr(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, w, n_valid, args.cpu_seconds)
+
+    workloads = None
+    if not args.no_workloads and world == 1:
+        del lay, graphs
+        torch.cuda.empty_cache()
+        workloads = {}
+        for name in ("tiny_4k", "llama8b_32k", "batch8_64k_b256", "qwen8b_128k_rope"):
+            if name == w.name:
+                continue
+            try:
+                workloads[name] = workload_line(name, args.workload_steps, 20, dev, peak)
+            except Exception as exc:  # noqa: BLE001 - a secondary line must not cost the headline
+                workloads[name] = {"error": f"{type(exc).__name__}: {exc}"}
+            torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
@@ -425,24 +559,28 @@ def run_hhr(args):
                 "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": n_valid,
                 "page": w.page, "P": w.P, "k": w.k, "bits": w.bits, "global_batch": w.B * world,
                 "seq_len": n_valid, "parallelism": f"replicas x{world} (independent units)",
-                "layers_cycled": L, "l2": f"inputs larger than L2: {L} layer instances cycled "
-                f"({alg * L / 2**20:.0f} MiB touched per cycle)", "launch": launch,
+                "layers_cycled": L, "l2": f"inputs larger than L2: {L} layer instances cycled, each with "
+                f"its own K, V, codes, metadata, R and W ({alg * L / 2**20:.0f} MiB touched per cycle)",
+                "launch": launch,
             },
             "keys_scored_per_s": agg["keys_scored_per_s"],
             "candidates_scored_per_s": candidates_per_step * world / (us_step * 1e-6),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "frac_vs_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                          "traffic": profiled_traffic(w.name), "peak_source": peak_kind,
                          "algorithmic_bytes": alg, "bytes_breakdown": parts,
                          "kernel": "decode_kernel<4,4,fused>"},
             "e2e": {"value": round(e2e_us, 3), "unit": UNIT,
                     "h2d_bytes_per_step": int(q_pin.numel() * q_pin.element_size()),
                     "d2h_bytes_per_step": int(out_pin.numel() * out_pin.element_size()),
-                    "steps": n_e2e, "how": "pinned q H2D + hhr_decode_step + out D2H + sync, per step"},
+                    "steps": n_e2e, "how": "hhr_decode_step_host per step: pinned q H2D + decode step + "
+                                           "out D2H + stream sync, one prepared ctypes call"},
             "gpu_launches": K,
             "planted_recall": recall,
             "clocks": clocks,
             "encode": encode_line(enc_ms, enc_flops, w.B * w.Hkv * n_valid),
+            "workloads": workloads,
             "cpu_baseline": cpu,
             "context": "pages' own numbers (A800, PyTorch): 3.30x decode and 2.83x end-to-end "
                        "speedup over dense attention at 128K, Llama-3.1-8B-Instruct",
@@ -450,7 +588,7 @@ def run_hhr(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
-        graphs.clear()
+        graphs = {}
         dist.destroy_process_group()
 
 

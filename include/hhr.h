@@ -202,6 +202,22 @@ int32_t hhr_decode_step(const hhr_dims* dims, const void* q, const float* R, con
                         int32_t* tok_idx, int32_t* n_sel, float* out, void* workspace,
                         size_t ws_bytes, void* stream);
 
+/*
+ * hhr_decode_step for a caller whose query and output live in host memory:
+ * copies q_host (bf16 [B][Hq][d]) into the device buffer q, runs the step,
+ * copies out (f32 [B][Hq][d]) back into out_host and waits for `stream`
+ * before returning (the only blocking decode call).  Host buffers should be
+ * pinned (page-locked) for the copies to be asynchronous DMA.  Other
+ * arguments as for hhr_decode_step; every check is made before anything is
+ * enqueued.  The paper has no counterpart: it is the end-to-end form of the
+ * decode step.
+ */
+int32_t hhr_decode_step_host(const hhr_dims* dims, const void* q_host, void* q, const float* R,
+                             const float* W, const uint32_t* codes, const void* meta, const void* K,
+                             const void* V, int32_t n_valid, int32_t P, int32_t k, float scale,
+                             int32_t* page_idx, int32_t* tok_idx, int32_t* n_sel, float* out,
+                             float* out_host, void* workspace, size_t ws_bytes, void* stream);
+
 /* Size of the scratch array hhr_decode_step_noalloc uses (4 MiB). */
 #define HHR_NOALLOC_SCRATCH_BYTES (4u << 20)
 
@@ -221,18 +237,29 @@ int32_t hhr_decode_step(const hhr_dims* dims, const void* q, const float* R, con
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture.
- *   - The call allocates nothing.  It enqueues a memset of the array's
- *     status word and counters, then the decode kernel.
+ *   - The call allocates nothing.  It checks every argument first (a rejected
+ *     call enqueues nothing and leaves the array alone), then enqueues a
+ *     memset of the array's per-unit counters and the decode kernel.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents: calls that may overlap on the GPU (different streams without
- *     ordering) race and give undefined results.  The bounded-wait status of
- *     this variant cannot be read back; it is cleared by the next call.
+ *     ordering) race and give undefined results.
+ *   - The array's status word records a bounded-wait timeout of any call
+ *     (outputs of that call are unspecified) and keeps it until
+ *     hhr_noalloc_read_status reads it.
  */
 int32_t hhr_decode_step_noalloc(const hhr_dims* dims, const void* q, const float* R,
                                 const float* W, const uint32_t* codes, const void* meta,
                                 const void* K, const void* V, int32_t n_valid, int32_t P,
                                 int32_t k, float scale, int32_t* page_idx, int32_t* tok_idx,
                                 int32_t* n_sel, float* out, void* stream);
+
+/*
+ * Status of hhr_decode_step_noalloc on the current device, as
+ * hhr_read_status gives it for a workspace: waits for `stream`, returns the
+ * scratch array's status word (HHR_OK or HHR_ERR_TIMEOUT) and clears it.
+ * Allocates nothing.  The paper has no counterpart.
+ */
+int32_t hhr_noalloc_read_status(void* stream);
 
 /*
  * Waits for `stream`, returns the workspace status word (HHR_OK or

@@ -57,9 +57,12 @@ _SIGS = {
                                  C.c_size_t, _P]),
     "hhr_decode_step": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32,
                                C.c_float, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "hhr_decode_step_host": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
+                                    _I32, C.c_float, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "hhr_decode_step_noalloc": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
                                        _I32, C.c_float, _P, _P, _P, _P, _P]),
     "hhr_read_status": (_I32, [_P, _P]),
+    "hhr_noalloc_read_status": (_I32, [_P]),
     "hhr_encode_status": (_I32, [_P]),
     "hhr_test_arm_timeout": (_I32, [_I32, C.c_uint64]),
 }
@@ -158,6 +161,41 @@ def hhr_decode_step(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page
                                  _ptr(workspace), ws_bytes, _stream(stream)), "hhr_decode_step")
 
 
+def hhr_decode_step_host(dims, q_host, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page_idx,
+                         tok_idx, n_sel, out, out_host, workspace=None, ws_bytes=None,
+                         stream=None) -> None:
+    """hhr_decode_step with the query and output in (pinned) host memory; blocks."""
+    ws_bytes = _nbytes(workspace) if ws_bytes is None and workspace is not None else (ws_bytes or 0)
+    _check(lib().hhr_decode_step_host(C.byref(dims), _ptr(q_host), _ptr(q), _ptr(R), _ptr(W),
+                                      _ptr(codes), _ptr(meta), _ptr(K), _ptr(V), n_valid, P, k, scale,
+                                      _ptr(page_idx), _ptr(tok_idx), _ptr(n_sel), _ptr(out),
+                                      _ptr(out_host), _ptr(workspace), ws_bytes, _stream(stream)),
+           "hhr_decode_step_host")
+
+
+def prepare(name, *args):
+    """A call of C function `name` with its arguments marshalled once (tensors
+    by data pointer, as above): returns a function that makes the call again
+    and raises HhrError on a non-zero status.  For repeated calls on the same
+    buffers (a decode loop), where per-call marshalling would dominate."""
+    fn = getattr(lib(), name)
+    conv = []
+    for a, t in zip(args, fn.argtypes):
+        if isinstance(a, hhr_dims):
+            conv.append(C.byref(a))
+        elif t is _P:
+            conv.append(C.c_void_p(_ptr(a)))
+        else:
+            conv.append(t(a))
+    conv = tuple(conv)
+
+    def call():
+        st = fn(*conv)
+        if st != HHR_OK:
+            raise HhrError(st, name)
+    return call
+
+
 def hhr_decode_step_noalloc(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page_idx,
                             tok_idx, n_sel, out, stream=None) -> None:
     """hhr_decode_step with the library's built-in scratch (no workspace)."""
@@ -172,6 +210,14 @@ def hhr_read_status(workspace, stream=None) -> int:
     st = lib().hhr_read_status(_ptr(workspace), _stream(stream))
     if st == HHR_ERR_CUDA:
         raise HhrError(st, "hhr_read_status")
+    return st
+
+
+def hhr_noalloc_read_status(stream=None) -> int:
+    """Status word of hhr_decode_step_noalloc's built-in scratch, cleared after reading."""
+    st = lib().hhr_noalloc_read_status(_stream(stream))
+    if st == HHR_ERR_CUDA:
+        raise HhrError(st, "hhr_noalloc_read_status")
     return st
 
 

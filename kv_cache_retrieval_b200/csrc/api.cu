@@ -242,7 +242,8 @@ static int32_t decode_common(const hhr_dims* dims, int mode, const void* q, cons
                              const void* V, const int32_t* tok_in, const int32_t* nsel_in,
                              int32_t n_valid, int32_t P, int32_t k, float scale, int32_t* page_idx,
                              int32_t* tok_idx, int32_t* n_sel, float* out, float* dbg_U,
-                             int32_t* dbg_D, void* workspace, size_t ws_bytes, void* stream) {
+                             int32_t* dbg_D, void* workspace, size_t ws_bytes, void* stream,
+                             bool check_only = false) {
   if (int32_t st = check_dims(dims)) return st;
   if (np_cap_of(dims) > HHR_MAX_PAGES) return HHR_ERR_UNSUPPORTED;
   if (k < 1 || !q) return HHR_ERR_INVALID_ARG;
@@ -263,6 +264,7 @@ static int32_t decode_common(const hhr_dims* dims, int mode, const void* q, cons
   std::memset(&a, 0, sizeof a);
   size_t smem = 0;
   if (int32_t st = plan_decode(dims, mode, n_valid, P, k, &a, &smem)) return st;
+  if (check_only) return HHR_OK;
   a.q = static_cast<const uint16_t*>(q);
   a.R = R;
   a.W = W;
@@ -316,6 +318,44 @@ int32_t hhr_decode_step(const hhr_dims* dims, const void* q, const float* R, con
   return decode_common(dims, kModeFused, q, R, W, codes, meta, K, V, nullptr, nullptr, n_valid, P,
                        k, scale, page_idx, tok_idx, n_sel, out, nullptr, nullptr, workspace,
                        ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace hhr {
+// Every check hhr_decode_step makes before it enqueues work, without
+// enqueuing any (the allocation-free variant validates before it touches its
+// shared scratch).
+int32_t decode_step_check(const hhr_dims* dims, const void* q, const float* R, const float* W,
+                          const uint32_t* codes, const void* meta, const void* K, const void* V,
+                          int32_t n_valid, int32_t P, int32_t k, float scale, int32_t* page_idx,
+                          int32_t* tok_idx, int32_t* n_sel, float* out, void* workspace,
+                          size_t ws_bytes) {
+  return decode_common(dims, kModeFused, q, R, W, codes, meta, K, V, nullptr, nullptr, n_valid, P,
+                       k, scale, page_idx, tok_idx, n_sel, out, nullptr, nullptr, workspace,
+                       ws_bytes, nullptr, true);
+}
+}  // namespace hhr
+
+extern "C" {
+
+int32_t hhr_decode_step_host(const hhr_dims* dims, const void* q_host, void* q, const float* R,
+                             const float* W, const uint32_t* codes, const void* meta, const void* K,
+                             const void* V, int32_t n_valid, int32_t P, int32_t k, float scale,
+                             int32_t* page_idx, int32_t* tok_idx, int32_t* n_sel, float* out,
+                             float* out_host, void* workspace, size_t ws_bytes, void* stream) {
+  if (!q_host || !out_host) return HHR_ERR_INVALID_ARG;
+  if (int32_t st = hhr::decode_step_check(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale,
+                                          page_idx, tok_idx, n_sel, out, workspace, ws_bytes))
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t qn = static_cast<size_t>(dims->B) * dims->Hq * dims->d;
+  if (cudaMemcpyAsync(q, q_host, qn * 2, cudaMemcpyHostToDevice, s) != cudaSuccess) return HHR_ERR_CUDA;
+  if (int32_t st = hhr_decode_step(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page_idx,
+                                   tok_idx, n_sel, out, workspace, ws_bytes, stream))
+    return st;
+  if (cudaMemcpyAsync(out_host, out, qn * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return HHR_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? HHR_OK : HHR_ERR_CUDA;
 }
 
 int32_t hhr_encode_status(void* stream) {

@@ -161,6 +161,13 @@ inline cudaError_t ensure_smem_limit(const void* kernel, size_t bytes, std::atom
   return e;
 }
 
+// hhr_decode_step's argument and size checks without launching (api.cu).
+int32_t decode_step_check(const hhr_dims* dims, const void* q, const float* R, const float* W,
+                          const uint32_t* codes, const void* meta, const void* K, const void* V,
+                          int32_t n_valid, int32_t P, int32_t k, float scale, int32_t* page_idx,
+                          int32_t* tok_idx, int32_t* n_sel, float* out, void* workspace,
+                          size_t ws_bytes);
+
 // Launchers (defined in decode.cu / encode.cu).  Return a cudaError_t.
 cudaError_t launch_decode(const DecodeArgs& a, int r, int bits, int mode, size_t smem_bytes,
                           cudaStream_t stream);

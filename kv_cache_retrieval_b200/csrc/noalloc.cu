@@ -50,13 +50,28 @@ extern "C" int32_t hhr_decode_step_noalloc(const hhr_dims* dims, const void* q, 
   if (need > HHR_NOALLOC_SCRATCH_BYTES) return HHR_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (int32_t st = scratch_address(&scratch)) return st;
-  // The status word and the per-unit counters must start at zero; the rest
-  // of the scratch is written before it is read within a call.
+  // every argument check first: a rejected call must not touch the scratch
+  // that a call still running on the GPU may be using
+  if (int32_t st = hhr::decode_step_check(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale,
+                                          page_idx, tok_idx, n_sel, out, scratch,
+                                          HHR_NOALLOC_SCRATCH_BYTES))
+    return st;
+  // The per-unit counters must start at zero (a timed-out call leaves them
+  // set); the status word is left as it is until hhr_noalloc_read_status
+  // reads it.  The rest of the scratch is written before it is read.
   const hhr::WsLayout L =
       hhr::ws_layout(dims->B * dims->Hkv, (dims->n_cap + dims->page - 1) / dims->page,
                      dims->Hq / dims->Hkv, dims->bits);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, L.U, s) != cudaSuccess) return HHR_ERR_CUDA;
+  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + L.counters, 0, L.U - L.counters, s) != cudaSuccess)
+    return HHR_ERR_CUDA;
   return hhr_decode_step(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page_idx, tok_idx,
                          n_sel, out, scratch, HHR_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int32_t hhr_noalloc_read_status(void* stream) {
+  void* scratch = nullptr;
+  if (int32_t st = scratch_address(&scratch)) return st;
+  // the status word is the scratch's first word, as in a caller workspace
+  return hhr_read_status(scratch, stream);
 }

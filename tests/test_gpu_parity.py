@@ -262,6 +262,30 @@ def test_timeout_hook_rejects_unknown_site():
         hhr.hhr_test_arm_timeout(7, 1000)
 
 
+def test_host_buffer_step_matches_device_step():
+    """hhr_decode_step_host (pinned host query in, host output back, blocking)
+    gives what hhr_decode_step gives, through a prepared call."""
+    from kv_cache_retrieval_b200 import _binding as Bnd
+    inp, codes, meta = case("llama_20k_ragged")
+    w = inp.w
+    d = Dev(inp)
+    d.load_state(codes, meta)
+    d.decode(0)
+    ref_out, ref_tok = _host(d.out).copy(), _host(d.tok_idx).copy()
+    q_pin = d.q[0].cpu().pin_memory()
+    out_pin = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(d.q[0])
+    d.out.fill_(float("nan"))
+    call = Bnd.prepare("hhr_decode_step_host", d.dims, q_pin, q_dev, d.R, d.W, d.codes, d.meta, d.K,
+                       d.V, w.N, d.P, d.k, d.scale, d.page_idx, d.tok_idx, d.n_sel, d.out, out_pin,
+                       d.ws, d.ws.numel(), torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):
+        call()
+        assert np.array_equal(out_pin.numpy(), ref_out)
+        assert np.array_equal(_host(d.tok_idx), ref_tok)
+    assert d.status() == hhr.HHR_OK
+
+
 # -------------------------------------------------------------- full sizes
 
 FULL_SAMPLES = {

@@ -41,6 +41,15 @@ def test_noalloc_step_matches_workspace_step_twice():
         assert torch.equal(n_sel, d.n_sel), f"call {step}: n_sel differs"
         err = float((out - d.out).abs().max().item())
         assert err <= ATTN_TOL, f"call {step}: max abs difference {err}"
+        assert hhr.hhr_noalloc_read_status() == hhr.HHR_OK
+    # a rejected call reports the error and leaves the scratch alone
+    st = Bnd.lib().hhr_decode_step_noalloc(C.byref(d.dims), None, d.R.data_ptr(), d.W.data_ptr(),
+                                           d.codes.data_ptr(), d.meta.data_ptr(), d.K.data_ptr(),
+                                           d.V.data_ptr(), w.N, d.P, d.k, d.scale,
+                                           page_idx.data_ptr(), tok_idx.data_ptr(),
+                                           n_sel.data_ptr(), out.data_ptr(), None)
+    assert st == hhr.HHR_ERR_INVALID_ARG
+    assert hhr.hhr_noalloc_read_status() == hhr.HHR_OK
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
