@@ -64,6 +64,12 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
   return old;
 }
 
+// Arrival on a unit barrier: release (the CTA's prior writes, made visible to
+// thread 0 by a CTA barrier, become visible before the count), no result.
+__device__ __forceinline__ void red_add_release(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(d), "l"(gmem_src) : "memory");
@@ -363,27 +369,77 @@ struct Smem {
   unsigned char* scratch;
 };
 
-// One warp: the merge weights of n partial softmax states of one head (in
-// shared memory).  State i has its running max at st[i * stride + d] and its
-// sum at st[i * stride + d + 1].  Writes wgt[i] = 2^(m_i - M) (M the largest
-// m_i; zero when every state is empty) and hdr = {M, sum_i wgt[i] l_i}.
-__device__ __forceinline__ void merge_weights(const float* st, int stride, int n, float* wgt, float* hdr) {
+// One warp merges n partial softmax states of one head; lane l takes the V
+// consecutive columns j0 + V l.  State i keeps its unnormalised outputs at
+// o[i * stride + column], its running max (base-2 logits) at ml[i * stride]
+// and its sum at ml[i * stride + 1]; an empty state has max -inf and sum 0.
+// With M = max_i m_i and weights w_i = 2^(m_i - M) (all zero when every state
+// is empty), res = sum_i w_i o_i over the lane's columns, and M and
+// L = sum_i w_i l_i in every lane.  The first kLoads states' outputs are
+// loaded at once (all in flight together; V = 4: 16-B loads, o, stride and
+// j0 multiples of 4 floats), the rest one by one; n <= 64.  kL2: the states
+// were written by other CTAs of this kernel, so they are read from L2.
+template <int kLoads, bool kL2, int V>
+__device__ __forceinline__ void merge_states(const float* o, const float* ml, int stride, int n, int j0,
+                                             float (&res)[V], float& M, float& L) {
+  static_assert(kLoads <= 32 && (V == 1 || V == 4), "lane i holds the weight of state i (and of 32 + i)");
   const int lane = threadIdx.x & 31;
-  float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, st[i * stride + kD]);
-#pragma unroll
-  for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o2));
-  float L = 0.f;
-  for (int i = lane; i < n; i += 32) {
-    const float w = (M == -INFINITY) ? 0.f : exp2f(st[i * stride + kD] - M);
-    wgt[i] = w;
-    L = fmaf(st[i * stride + kD + 1], w, L);
+  auto ld = [](const float* p) { return kL2 ? __ldcg(p) : *p; };
+  auto ldv = [&](int i, float (&dst)[V]) {
+    const float* p = o + i * stride + j0 + V * lane;
+    if constexpr (V == 4) {
+      const float4 t = kL2 ? __ldcg(reinterpret_cast<const float4*>(p)) : *reinterpret_cast<const float4*>(p);
+      dst[0] = t.x;
+      dst[1] = t.y;
+      dst[2] = t.z;
+      dst[3] = t.w;
+    } else {
+      dst[0] = ld(p);
+    }
+  };
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  if (lane < n) {
+    m0 = ld(ml + lane * stride);
+    l0 = ld(ml + lane * stride + 1);
   }
+  if (lane + 32 < n) {
+    m1 = ld(ml + (lane + 32) * stride);
+    l1 = ld(ml + (lane + 32) * stride + 1);
+  }
+  float ov[kLoads][V];
 #pragma unroll
-  for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o2);
-  if (lane == 0) {
-    hdr[0] = M;
-    hdr[1] = L;
+  for (int i = 0; i < kLoads; ++i) {
+    if (i < n) {
+      ldv(i, ov[i]);
+    } else {
+#pragma unroll
+      for (int v = 0; v < V; ++v) ov[i][v] = 0.f;
+    }
+  }
+  float mx = fmaxf(m0, m1);
+#pragma unroll
+  for (int o2 = 16; o2 >= 1; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o2));
+  const float w0 = (mx == -INFINITY) ? 0.f : exp2f(m0 - mx);
+  const float w1 = (mx == -INFINITY) ? 0.f : exp2f(m1 - mx);
+  float ls = fmaf(l0, w0, l1 * w1);
+#pragma unroll
+  for (int o2 = 16; o2 >= 1; o2 >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, o2);
+  M = mx;
+  L = ls;
+#pragma unroll
+  for (int v = 0; v < V; ++v) res[v] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kLoads; ++i) {
+    const float w = __shfl_sync(0xFFFFFFFFu, w0, i);
+#pragma unroll
+    for (int v = 0; v < V; ++v) res[v] = fmaf(ov[i][v], w, res[v]);
+  }
+  for (int i = kLoads; i < n; ++i) {   // warp-uniform trip count
+    const float w = __shfl_sync(0xFFFFFFFFu, i < 32 ? w0 : w1, i & 31);
+    float t[V];
+    ldv(i, t);
+#pragma unroll
+    for (int v = 0; v < V; ++v) res[v] = fmaf(t[v], w, res[v]);
   }
 }
 
@@ -561,29 +617,22 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   }
   __syncthreads();
 
+  // the CTA's state: warp item = (head h, 32-column block) merges the 16
+  // warp states of its columns.  Stored as [r][d] outputs, then (max, sum)
+  // per head, so that each head's outputs are 16-B aligned.
   constexpr int PS = part_stride(RG);
   float* part = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * PS;
-  {
-    // weights e^(m_w - M) of the 16 warp states of each head (warp h does
-    // head h), then thread (h, j) combines the outputs with them
-    float* wgt = mer + NWARPS * RG * (kD + 2);   // [RG][NWARPS]
-    float* hdr = wgt + NWARPS * RG;              // [RG][2]: M, sum of weighted l
-    if (warp < RG) merge_weights(mer + warp * (kD + 2), RG * (kD + 2), NWARPS, wgt + warp * NWARPS, hdr + 2 * warp);
-    __syncthreads();
-    for (int oi = tid; oi < RG * kD; oi += NT) {
-      const int h = oi / kD, j = oi % kD;
-      float O = 0.f;
-#pragma unroll 4
-      for (int w = 0; w < NWARPS; ++w) O = fmaf(mer[(w * RG + h) * (kD + 2) + j], wgt[h * NWARPS + w], O);
-      const float L = hdr[2 * h + 1];
-      if (a.C == 1) {
-        a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
-      } else {
-        part[h * (kD + 2) + j] = O;
-        if (j == 0) {
-          part[h * (kD + 2) + kD] = hdr[2 * h];
-          part[h * (kD + 2) + kD + 1] = L;
-        }
+  for (int item = warp; item < RG * (kD / 32); item += NWARPS) {
+    const int h = item / (kD / 32), j0 = (item % (kD / 32)) * 32;
+    float M, L, O[1];
+    merge_states<NWARPS, false, 1>(mer + h * (kD + 2), mer + h * (kD + 2) + kD, RG * (kD + 2), NWARPS, j0, O, M, L);
+    if (a.C == 1) {
+      a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j0 + lane] = (L > 0.f) ? O[0] / L : 0.f;
+    } else {
+      part[h * kD + j0 + lane] = O[0];
+      if (lane == 0) {
+        part[RG * kD + 2 * h] = M;
+        part[RG * kD + 2 * h + 1] = L;
       }
     }
   }
@@ -601,26 +650,17 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
   __syncthreads();
   if (!s_int[0]) return;
   if (a.C > 1) {
-    // the C partial states of the unit, copied from L2 in one batch of 16-B
-    // chunks (PS is a multiple of 4 floats); then weights by one warp per
-    // head, and thread (h, j) combines column j of head h
+    // the C partial states of the unit, straight from L2: one warp per
+    // head, four columns a lane, the loads of up to 20 states all in flight
+    // at once (16-B loads: many single-float loads in flight from one SM
+    // take several L2 round trips)
     const float* parts = a.wsPart + static_cast<size_t>(unit * kMaxCtasPerUnit) * PS;
-    float* sp = reinterpret_cast<float*>(scratch);    // [C][PS]
-    float* wgt = sp + a.C * PS;                       // [RG][C]
-    float* hdr = wgt + a.C * RG;                      // [RG][2]
-    for (int i = tid; i < a.C * PS / 4; i += NT) cp_async16(sp + 4 * i, parts + 4 * i);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    if (warp < RG) merge_weights(sp + warp * (kD + 2), PS, a.C, wgt + warp * a.C, hdr + 2 * warp);
-    __syncthreads();
-    for (int oi = tid; oi < RG * kD; oi += NT) {
-      const int h = oi / kD, j = oi % kD;
-      float O = 0.f;
-#pragma unroll 6
-      for (int cc = 0; cc < a.C; ++cc) O = fmaf(sp[cc * PS + h * (kD + 2) + j], wgt[h * a.C + cc], O);
-      const float L = hdr[2 * h + 1];
-      a.out[(static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + j] = (L > 0.f) ? O / L : 0.f;
+    for (int h = warp; h < RG; h += NWARPS) {
+      float M, L, O[4];
+      merge_states<20, true, 4>(parts + h * kD, parts + RG * kD + 2 * h, PS, a.C, 0, O, M, L);
+      float* dst = a.out + (static_cast<size_t>(b) * a.Hq + g * RG + h) * kD + 4 * lane;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) dst[v] = (L > 0.f) ? O[v] / L : 0.f;
     }
   }
   if (tid == 0) atomicExch(a.counters + unit, 0u);
@@ -630,11 +670,6 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
 template <int RG, int WORDS, int MODE>
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  // Launched as a programmatic dependent of the previous kernel on the
-  // stream: wait here, before any global memory access, until that kernel
-  // has completed and its writes are visible.  Only the launch itself
-  // overlaps; no work of two steps does.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int s_int[NWARPS + 16];
   __shared__ int s_scan1[NWARPS];
   __shared__ int s_aux[264];  // distance totals (<= 257 bins)
@@ -656,6 +691,22 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
   __shared__ __align__(8) unsigned long long s_rwbar;                       // W staging
   const uint32_t rw_addr = smem_addr(&s_rwbar);
   uint32_t rw_seq = 0;  // W phases used so far
+  float* sRW = reinterpret_cast<float*>(S.scratch + NWARPS * kLaneSlots * 512);  // R / W staging
+  // thread 0: one bulk copy of the d x d rotation of KV head g into sRW
+  auto issue_r = [&](int g) {
+    // the storage may last have been touched by generic-proxy accesses
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
+    bulk_g2s_keep(smem_addr(sRW), a.R + static_cast<size_t>(g) * kD * kD, kD * kD * sizeof(float), rw_addr);
+  };
+  const int unit0 = blockIdx.x / a.C;
+  // this CTA's page range and its warp's share of it (the same for every unit)
+  const int pb = c * a.NP / a.C;      // c * NP < 2^20 (NP <= HHR_MAX_PAGES)
+  const int pe = (c + 1) * a.NP / a.C;
+  const int my_pages = pe - pb;
+  const int wpb = pb + my_pages * warp / NWARPS;
+  const int wpe = pb + my_pages * (warp + 1) / NWARPS;
+  const int w_pages = wpe - wpb;
   if (tid == 0) {
     mbar_init(rw_addr, 1u);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -664,9 +715,17 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
     // the B operand's unused columns (fourth term of each head, absent heads) stay zero
     for (int i = tid; i < 8 * ((RG * 4 + 7) / 8) * 2 * kD; i += NT) S.qb[i] = 0;
   }
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: the set-up above touches no global memory and may overlap that
+  // kernel's tail; from here on, its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the first unit's R goes out before anything else: the query transform
+  // waits on it
+  if constexpr (MODE != kModeAttend)
+    if (tid == 0 && unit0 < a.units) issue_r(unit0 % a.Hkv);
   __syncthreads();
 
-  for (int unit = blockIdx.x / a.C; unit < a.units; unit += a.grid_units) {
+  for (int unit = unit0; unit < a.units; unit += a.grid_units) {
     const int b = unit / a.Hkv, g = unit % a.Hkv;
 
     uint32_t* ctr = a.counters + unit;
@@ -675,8 +734,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
 
     if constexpr (MODE == kModeAttend) {
       const int n = a.nsel_in[unit];
-      const int s0 = static_cast<int>(static_cast<long long>(c) * n / a.C);
-      const int s1 = static_cast<int>(static_cast<long long>(c + 1) * n / a.C);
+      const int s0 = c * n / a.C;         // c * n < 2^26 (n <= C * kMaxTokensPerCta)
+      const int s1 = (c + 1) * n / a.C;
       const int32_t* src = a.tok_in + static_cast<size_t>(unit) * a.k;
 #pragma unroll 8
       for (int i = s0 + tid; i < s1; i += NT) S.sel[i - s0] = src[i];
@@ -691,11 +750,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // pages of each warp at once, the rest of the ring -- which shares its
       // storage with R -- as soon as q~ = q R is formed.  W follows by bulk
       // copy on an mbarrier once the ring has drained.
-      const long long pb = static_cast<long long>(c) * a.NP / a.C;
-      const long long pe = static_cast<long long>(c + 1) * a.NP / a.C;
-      const int my_pages = static_cast<int>(pe - pb);
-      float* sRW = reinterpret_cast<float*>(S.scratch + NWARPS * kLaneSlots * 512);
-      const float* Rg = a.R + static_cast<size_t>(g) * kD * kD;
       const float* Wg = a.W + static_cast<size_t>(g) * kD * BITS;
       auto issue_w = [&](int half_w) {  // thread 0 only: 128 columns of W
         // the storage was last touched by generic-proxy copies and loads
@@ -722,9 +776,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // barrier is involved.  Slot s of warp w is the 512 B at
       // (s * NWARPS + w) * 512: slots [0, kLaneSlots) lie below the R / W
       // buffer, slots [kLaneSlots, kRingSlots) inside it.
-      const long long wpb = pb + static_cast<long long>(my_pages) * warp / NWARPS;
-      const long long wpe = pb + static_cast<long long>(my_pages) * (warp + 1) / NWARPS;
-      const int w_pages = static_cast<int>(wpe - wpb);
       constexpr int PPG = 8;                        // pages per ring group; an A tile is two groups
       constexpr int G0 = 1;                         // groups in flight while q~ is formed (A/B: 1 beats 0 and 2)
       constexpr int GR = kRingSlots / PPG;          // groups in flight afterwards
@@ -752,13 +803,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         cp_async_commit();
       };
 
-      // R alone first, one bulk copy: requested together with the metadata
-      // it would land only with the whole first burst
-      if (tid == 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_expect_tx(rw_addr, kD * kD * sizeof(float));
-        bulk_g2s_keep(smem_addr(sRW), Rg, kD * kD * sizeof(float), rw_addr);
-      }
+      // R alone first, one bulk copy (the first unit's went out at the
+      // kernel's start): requested together with the metadata it would land
+      // only with the whole first burst
+      if (tid == 0 && unit != unit0) issue_r(g);
       // queries of the group, as float (raw) -- q~ is derived from these
       for (int i = tid; i < RG * kD; i += NT) S.qf[i] = __uint_as_float(static_cast<uint32_t>(qg[i]) << 16);
       if (!wait_rw()) {
@@ -859,7 +907,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
             const int pl = ti * 16 + g8 + 8 * hr;
             if (pl < w_pages) {
               const float u = hr ? u1 : u0;
-              const long long pg = wpb + pl;
+              const int pg = wpb + pl;
               wsU_u[pg] = u;
               if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
               lmin = fminf(lmin, u);
@@ -901,7 +949,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         issue_w(0);
         // unit barrier 1: arrive now (the release covers the CTA's U through
         // the CTA barrier above), wait after the query codes
-        atom_add_acq_rel(ctr, 1u);
+        red_add_release(ctr, 1u);
       }
       // query codes (Eq. 10 + sign) from W in shared memory, 128 columns at
       // a time, while the other CTAs of the unit finish their bounds
@@ -1139,7 +1187,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         // loads then hit L2 (a hint only; rows clamped to the codes buffer)
         const size_t row_bytes = static_cast<size_t>(WORDS) * 4;
         const char* cbase = reinterpret_cast<const char*>(a.codes + static_cast<size_t>(unit) * a.n_cap * WORDS);
-        for (long long p = pb + tid; p < pe; p += NT) {
+        for (int p = pb + tid; p < pe; p += NT) {
           if ((sBits[p >> 5] >> (p & 31)) & 1u) {
             const size_t b0 = static_cast<size_t>(p) * a.page * row_bytes;
             const size_t b1 = min(static_cast<size_t>(p + 1) * a.page, static_cast<size_t>(a.n_cap)) * row_bytes;
@@ -1149,8 +1197,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       }
 
       // ---------------------------------------------------------- phase 3
-      const int ks = static_cast<int>(static_cast<long long>(c) * Pk / a.C);
-      const int ke = static_cast<int>(static_cast<long long>(c + 1) * Pk / a.C);
+      const int ks = c * Pk / a.C;
+      const int ke = (c + 1) * Pk / a.C;
       {
         // thread t owns bitmap words [t*wpt, (t+1)*wpt)
         const int wpt = (nwords + NT - 1) / NT;
@@ -1233,7 +1281,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // unit barrier 2 (the release by thread 0 covers the CTA's histogram
       // row through the CTA barrier)
       __syncthreads();
-      if (tid == 0) atom_add_acq_rel(ctr, 1u);
+      if (tid == 0) red_add_release(ctr, 1u);
       if (!unit_wait(ctr, 2u * static_cast<uint32_t>(a.C) + (a.test_extra_stage == 2 ? 1u : 0u), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 5
@@ -1251,56 +1299,88 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         cp_async_wait<0>();
       }
       __syncthreads();
-      // distance totals tot[v] = sum over the CTAs (thread v); one block-wide
-      // exclusive scan of them gives k_eff, the threshold distance T (the
-      // k_eff-th smallest) and how many tokens at T are still needed
-      int* sbe = sHA + a.C * (BITS + 1);                 // [C][2]: below T, at T
-      if (tid == 0) {
-        s_misc[4] = 0;
-        s_misc[5] = -1;
+      // Every CTA row's exclusive prefix over the distances (warp per row:
+      // lane l owns bins [VPL l, VPL l + VPL), bin BITS + 1 empty, so that
+      // pre[cc][BITS + 1] is the row's total) and the unit totals tot[v]
+      // (thread v); then warp 0 alone finds the threshold distance T (the
+      // k_eff-th smallest), how many tokens at T are still needed, and each
+      // CTA's tie quota and output offset in CTA order.
+      constexpr int VPL = (BITS + 2 + 31) / 32;
+      int* sPre = sHA + a.C * (BITS + 1);                // [C][BITS + 2]
+      int* sTot = sPre + a.C * (BITS + 2);               // [BITS + 1]
+      for (int cc = warp; cc < a.C; cc += NWARPS) {
+        const int* row = sHA + cc * (BITS + 1);
+        int hv[VPL], loc = 0;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) {
+          const int v = lane * VPL + e;
+          hv[e] = v <= BITS ? row[v] : 0;
+          loc += hv[e];
+        }
+        int incl = loc;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+          const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
+          if (lane >= o2) incl += y;
+        }
+        int run = incl - loc;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) {
+          const int v = lane * VPL + e;
+          if (v <= BITS + 1) sPre[cc * (BITS + 2) + v] = run;
+          run += hv[e];
+        }
       }
-      {
+      if (tid <= BITS) {
         int x = 0;
-        if (tid <= BITS) {
 #pragma unroll 6
-          for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * (BITS + 1) + tid];
-        }
-        int total;
-        const int excl = block_excl_scan(x, s_scan, &total);
-        const int k_eff = min(a.k, total);
-        if (x > 0 && excl < k_eff && excl + x >= k_eff) {   // exactly one thread
-          s_misc[5] = tid;
-          s_misc[4] = k_eff - excl;
-        }
-        if (tid == 0) s_misc[6] = k_eff;
+        for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * (BITS + 1) + tid];
+        sTot[tid] = x;
       }
       __syncthreads();
-      {
-        // per-CTA tokens below T / at T: a half-warp per CTA row
-        const int T = s_misc[5];
-        // warp-uniform trip count: each warp takes rows base and base + 1
-        for (int base = warp * 2; base < a.C; base += NT / 16) {
-          const int cc = base + (lane >> 4), part = lane & 15;
-          const bool row_ok = cc < a.C;
-          int below = 0;
-          if (row_ok)
-            for (int v = part; v < T; v += 16) below += sHA[cc * (BITS + 1) + v];
+      if (warp == 0) {
+        int xv[VPL], loc = 0;
 #pragma unroll
-          for (int o2 = 8; o2 >= 1; o2 >>= 1) below += __shfl_xor_sync(0xFFFFFFFFu, below, o2);
-          if (row_ok && part == 0) {
-            sbe[2 * cc] = below;
-            sbe[2 * cc + 1] = T >= 0 ? sHA[cc * (BITS + 1) + T] : 0;
+        for (int e = 0; e < VPL; ++e) {
+          const int v = lane * VPL + e;
+          xv[e] = v <= BITS ? sTot[v] : 0;
+          loc += xv[e];
+        }
+        int incl = loc;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+          const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
+          if (lane >= o2) incl += y;
+        }
+        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const int k_eff = min(a.k, total);
+        // the lane whose bins hold the k_eff-th smallest distance
+        int T = -1, needT = 0;
+        if (incl - loc < k_eff && incl >= k_eff) {
+          int run = incl - loc;
+#pragma unroll
+          for (int e = 0; e < VPL; ++e) {
+            if (run < k_eff && run + xv[e] >= k_eff) {
+              T = lane * VPL + e;
+              needT = k_eff - run;
+            }
+            run += xv[e];
           }
         }
-      }
-      __syncthreads();
-      if (warp == 0) {  // in CTA order: tie quota and output offset of each CTA
-        const int needT = s_misc[4];
+        const unsigned own = __ballot_sync(0xFFFFFFFFu, T >= 0);
+        if (own) {
+          const int src = __ffs(own) - 1;
+          T = __shfl_sync(0xFFFFFFFFu, T, src);
+          needT = __shfl_sync(0xFFFFFFFFu, needT, src);
+        }
         int pre_eq = 0, off = 0;
-        for (int c0 = 0; c0 < a.C; c0 += 32) {
+        for (int c0 = 0; c0 < a.C; c0 += 32) {   // CTAs in order: tie quota and output offset
           const int cc = c0 + lane;
-          const int below = cc < a.C ? sbe[2 * cc] : 0;
-          const int eq = cc < a.C ? sbe[2 * cc + 1] : 0;
+          int below = 0, eq = 0;
+          if (cc < a.C && T >= 0) {
+            below = sPre[cc * (BITS + 2) + T];
+            eq = sPre[cc * (BITS + 2) + T + 1] - below;
+          }
           int eq_in = eq;
 #pragma unroll
           for (int o2 = 1; o2 < 32; o2 <<= 1) {
@@ -1322,6 +1402,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           }
           pre_eq += __shfl_sync(0xFFFFFFFFu, eq_in, 31);
           off += __shfl_sync(0xFFFFFFFFu, sel_in, 31);
+        }
+        if (lane == 0) {
+          s_misc[5] = T;
+          s_misc[6] = k_eff;
         }
       }
       __syncthreads();

@@ -112,14 +112,13 @@ inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, 
         + sizeof(uint32_t) * align_up(((size_t)NP + 31) / 32, 4)  // kept bitmap
         + 2 * (sizeof(float) + sizeof(int)) * kCandMax       // boundary candidates, 2 levels
         + sizeof(float) * 2 * (kDecodeThreads / 32);          // level-2 min / max
-    hist = sizeof(int) * ((size_t)C * (bits + 1) + 2 * (size_t)C) + 16;
+    // distance histograms, their row prefixes, the unit totals (+ copy rounding)
+    hist = sizeof(int) * ((size_t)C * (bits + 1) + (size_t)C * (bits + 2) + (bits + 1)) + 16;
   }
   if (mode != kModeSelect) {
     // per warp: K and V of 16 tokens; then the 16-row query tile
     const size_t ring = (size_t)(kDecodeThreads / 32) * 2 * 16 * 2 * kD + 16 * 2 * kD;
-    size_t merge = sizeof(float) * ((kDecodeThreads / 32) * (size_t)r * (kD + 2) + (kDecodeThreads / 32) * (size_t)r + 2 * (size_t)r);
-    const size_t parts = sizeof(float) * ((size_t)C * part_stride(r) + (size_t)C * r + 2 * (size_t)r);  // final merge
-    merge = merge > parts ? merge : parts;
+    const size_t merge = sizeof(float) * (kDecodeThreads / 32) * (size_t)r * (kD + 2);  // the warps' states
     attn = ring > merge ? ring : merge;
   }
   size_t m = sel > hist ? sel : hist;
