@@ -31,6 +31,11 @@
 //      ties go to the lower token index.  No sink/local tokens are forced in.
 //  R7  Attention over the selected keys is softmax(scale * q.k) V with the
 //      original (unrotated) keys; Eq. 4 shows the logits are unchanged by R.
+// Variants (flags of the *_v / *_f32 / *_agg entry points):
+//  V1  float32 page metadata: l and u kept exactly as the float32 extrema of
+//      the rotated keys (no rounding), instead of R1's outward bf16.
+//  V2  GQA-sum: the token distance is the sum over G(g) of Eq. 2, instead of
+//      R4's min (the paper does not treat grouped heads; both readings fit).
 
 #include <algorithm>
 #include <cmath>
@@ -71,6 +76,9 @@ uint16_t bf16_toward_pos_inf(float f) {
   if ((u & 0xFFFFu) == 0) return t;
   return (u >> 31) ? t : static_cast<uint16_t>(t + 1);
 }
+
+double meta_value(uint16_t h) { return widen_bf16(h); }
+double meta_value(float f) { return static_cast<double>(f); }
 
 int bit_count(uint32_t x) {
   int c = 0;
@@ -153,6 +161,28 @@ void hhro_page_meta(const float* kt, int64_t t0, int64_t n_valid, int32_t d, int
   }
 }
 
+// Variant V1 of the metadata above: the same extrema, kept in float32 as
+// computed (no rounding).
+void hhro_page_meta_f32(const float* kt, int64_t t0, int64_t n_valid, int32_t d, int32_t page,
+                        int64_t p_begin, int64_t p_end, float* meta) {
+  for (int64_t p = p_begin; p < p_end; ++p) {
+    const int64_t n0 = p * page;
+    const int64_t n1 = std::min<int64_t>(n0 + page, n_valid);
+    if (n1 <= n0) continue;
+    for (int j = 0; j < d; ++j) {
+      float lo = std::numeric_limits<float>::infinity();
+      float hi = -std::numeric_limits<float>::infinity();
+      for (int64_t n = n0; n < n1; ++n) {
+        const float v = kt[(n - t0) * d + j];
+        lo = std::min(lo, v);
+        hi = std::max(hi, v);
+      }
+      meta[(p * 2 + 0) * d + j] = lo;
+      meta[(p * 2 + 1) * d + j] = hi;
+    }
+  }
+}
+
 // Key encoding of one (sequence, KV head) for the keys [n_begin, n_end):
 // codes of those keys (Eq. 10 + sign) and the metadata of every page they
 // touch, recomputed from all keys [p*S, min((p+1)*S, n_end)) of that page
@@ -174,6 +204,22 @@ int64_t hhro_encode_unit(const uint16_t* K, int64_t n_begin, int64_t n_end, int3
                            codes + n_begin * words, nullptr);
 }
 
+// hhro_encode_unit with float32 metadata (variant V1).
+int64_t hhro_encode_unit_f32(const uint16_t* K, int64_t n_begin, int64_t n_end, int32_t d,
+                             int32_t bits, int32_t page, const float* R, const float* W,
+                             uint32_t* codes, float* meta) {
+  if (n_end <= n_begin) return 0;
+  const int64_t p0 = n_begin / page;
+  const int64_t p1 = (n_end - 1) / page + 1;
+  const int64_t t0 = p0 * page;
+  std::vector<float> kt(static_cast<size_t>((n_end - t0) * d));
+  hhro_rotate(K + t0 * d, n_end - t0, d, R, kt.data());
+  hhro_page_meta_f32(kt.data(), t0, n_end, d, page, p0, p1, meta);
+  const int words = bits / 32;
+  return hhro_project_sign(K + n_begin * d, n_end - n_begin, d, bits, W,
+                           codes + n_begin * words, nullptr);
+}
+
 // Query side of Eq. 4 (q~ = q R) and of Eq. 10 + sign, for the r query heads
 // of one KV group.  Returns the ambiguous-sign count of the query codes.
 int64_t hhro_query_prep(const uint16_t* q, int32_t r, int32_t d, int32_t bits,
@@ -186,18 +232,22 @@ int64_t hhro_query_prep(const uint16_t* q, int32_t r, int32_t d, int32_t bits,
 // the float32 q~ and the widened bf16 bounds; the group score is the max over
 // the r heads (reading R4).  Uh (nullable) receives the per-head values
 // [r][np].
-void hhro_page_bounds(const float* qt, int32_t r, int32_t d, const uint16_t* meta, int64_t np,
-                      double* U, double* Uh) {
+}  // extern "C"
+
+namespace {
+template <typename MetaT>
+void page_bounds(const float* qt, int32_t r, int32_t d, const MetaT* meta, int64_t np, double* U,
+                 double* Uh) {
   for (int64_t p = 0; p < np; ++p) {
-    const uint16_t* lo = meta + (p * 2 + 0) * d;
-    const uint16_t* hi = meta + (p * 2 + 1) * d;
+    const MetaT* lo = meta + (p * 2 + 0) * d;
+    const MetaT* hi = meta + (p * 2 + 1) * d;
     double best = -std::numeric_limits<double>::infinity();
     for (int h = 0; h < r; ++h) {
       double s = 0.0;
       for (int j = 0; j < d; ++j) {
         const double qj = static_cast<double>(qt[h * d + j]);
-        const double a = qj * widen_bf16(lo[j]);
-        const double b = qj * widen_bf16(hi[j]);
+        const double a = qj * meta_value(lo[j]);
+        const double b = qj * meta_value(hi[j]);
         s += std::max(a, b);
       }
       if (Uh) Uh[h * np + p] = s;
@@ -205,6 +255,20 @@ void hhro_page_bounds(const float* qt, int32_t r, int32_t d, const uint16_t* met
     }
     U[p] = best;
   }
+}
+}  // namespace
+
+extern "C" {
+
+void hhro_page_bounds(const float* qt, int32_t r, int32_t d, const uint16_t* meta, int64_t np,
+                      double* U, double* Uh) {
+  page_bounds(qt, r, d, meta, np, U, Uh);
+}
+
+// Eq. 3 on float32 metadata (variant V1).
+void hhro_page_bounds_f32(const float* qt, int32_t r, int32_t d, const float* meta, int64_t np,
+                          double* U, double* Uh) {
+  page_bounds(qt, r, d, meta, np, U, Uh);
 }
 
 // Page retention (§3.3.1 after Eq. 3, readings R5): indices of the
@@ -227,9 +291,10 @@ int64_t hhro_top_largest(const double* s, int64_t n, int64_t m, int32_t* out) {
 // query codes and the code of every valid token of the kept pages; the group
 // distance is the min over the r heads (reading R4).  D[slot*S + t] is the
 // distance of token pages[slot]*S + t, or -1 where that token is >= n_valid.
-void hhro_hamming(const uint32_t* qcode, int32_t r, int32_t words, const uint32_t* codes,
-                  const int32_t* pages, int64_t n_pages, int32_t page, int64_t n_valid,
-                  int32_t* D) {
+// agg = 0: min over the heads (R4); agg = 1: sum over the heads (V2).
+void hhro_hamming_agg(const uint32_t* qcode, int32_t r, int32_t words, const uint32_t* codes,
+                      const int32_t* pages, int64_t n_pages, int32_t page, int64_t n_valid,
+                      int32_t agg, int32_t* D) {
   for (int64_t slot = 0; slot < n_pages; ++slot) {
     for (int t = 0; t < page; ++t) {
       const int64_t n = static_cast<int64_t>(pages[slot]) * page + t;
@@ -237,15 +302,22 @@ void hhro_hamming(const uint32_t* qcode, int32_t r, int32_t words, const uint32_
         D[slot * page + t] = -1;
         continue;
       }
-      int best = std::numeric_limits<int>::max();
+      int best = std::numeric_limits<int>::max(), total = 0;
       for (int h = 0; h < r; ++h) {
         int dist = 0;
         for (int w = 0; w < words; ++w) dist += bit_count(qcode[h * words + w] ^ codes[n * words + w]);
         best = std::min(best, dist);
+        total += dist;
       }
-      D[slot * page + t] = best;
+      D[slot * page + t] = agg ? total : best;
     }
   }
+}
+
+void hhro_hamming(const uint32_t* qcode, int32_t r, int32_t words, const uint32_t* codes,
+                  const int32_t* pages, int64_t n_pages, int32_t page, int64_t n_valid,
+                  int32_t* D) {
+  hhro_hamming_agg(qcode, r, words, codes, pages, n_pages, page, n_valid, 0, D);
 }
 
 // Token selection (§3.3.2 inference + Top-K of §4.1, reading R6): among the
@@ -308,12 +380,14 @@ void hhro_attend(const uint16_t* q, int32_t r, int32_t d, const uint16_t* K, con
 // page_idx [P], tok_idx [k], D [P*S] (nullable), U [ceil(n_valid/S)]
 // (nullable).  Returns the number of selected tokens; *q_ambiguous receives
 // the ambiguous-sign count of the query codes.
-int64_t hhro_decode_unit(const uint16_t* q, int32_t r, int32_t d, int32_t bits, int32_t page,
-                         const float* R, const float* W, const uint32_t* codes,
-                         const uint16_t* meta, const uint16_t* K, const uint16_t* V,
-                         int64_t n_valid, int64_t P, int64_t k, double scale,
-                         int32_t* page_idx, int32_t* tok_idx, double* U, int32_t* D,
-                         float* out, int64_t* q_ambiguous) {
+// flags: bit 0 = float32 metadata (V1; meta is float [..][2][d]), bit 1 =
+// GQA-sum distances (V2).  hhro_decode_unit is flags = 0.
+int64_t hhro_decode_unit_v(const uint16_t* q, int32_t r, int32_t d, int32_t bits, int32_t page,
+                           const float* R, const float* W, const uint32_t* codes,
+                           const void* meta, const uint16_t* K, const uint16_t* V,
+                           int64_t n_valid, int64_t P, int64_t k, double scale, int32_t flags,
+                           int32_t* page_idx, int32_t* tok_idx, double* U, int32_t* D,
+                           float* out, int64_t* q_ambiguous) {
   const int words = bits / 32;
   std::vector<float> qt(static_cast<size_t>(r) * d);
   std::vector<uint32_t> qcode(static_cast<size_t>(r) * words);
@@ -322,7 +396,10 @@ int64_t hhro_decode_unit(const uint16_t* q, int32_t r, int32_t d, int32_t bits, 
 
   const int64_t np = (n_valid + page - 1) / page;
   std::vector<double> Ubuf(static_cast<size_t>(np));
-  hhro_page_bounds(qt.data(), r, d, meta, np, Ubuf.data(), nullptr);
+  if (flags & 1)
+    hhro_page_bounds_f32(qt.data(), r, d, static_cast<const float*>(meta), np, Ubuf.data(), nullptr);
+  else
+    hhro_page_bounds(qt.data(), r, d, static_cast<const uint16_t*>(meta), np, Ubuf.data(), nullptr);
   if (U)
     for (int64_t p = 0; p < np; ++p) U[p] = Ubuf[p];
 
@@ -331,7 +408,8 @@ int64_t hhro_decode_unit(const uint16_t* q, int32_t r, int32_t d, int32_t bits, 
   for (int64_t i = 0; i < P; ++i) page_idx[i] = i < n_kept ? kept[i] : -1;
 
   std::vector<int32_t> Dbuf(static_cast<size_t>(n_kept) * page);
-  hhro_hamming(qcode.data(), r, words, codes, kept.data(), n_kept, page, n_valid, Dbuf.data());
+  hhro_hamming_agg(qcode.data(), r, words, codes, kept.data(), n_kept, page, n_valid,
+                   (flags & 2) ? 1 : 0, Dbuf.data());
   if (D)
     for (int64_t i = 0; i < P * page; ++i) D[i] = i < n_kept * page ? Dbuf[i] : -1;
 
@@ -341,6 +419,16 @@ int64_t hhro_decode_unit(const uint16_t* q, int32_t r, int32_t d, int32_t bits, 
 
   if (out) hhro_attend(q, r, d, K, V, sel.data(), n_sel, scale, out);
   return n_sel;
+}
+
+int64_t hhro_decode_unit(const uint16_t* q, int32_t r, int32_t d, int32_t bits, int32_t page,
+                         const float* R, const float* W, const uint32_t* codes,
+                         const uint16_t* meta, const uint16_t* K, const uint16_t* V,
+                         int64_t n_valid, int64_t P, int64_t k, double scale,
+                         int32_t* page_idx, int32_t* tok_idx, double* U, int32_t* D,
+                         float* out, int64_t* q_ambiguous) {
+  return hhro_decode_unit_v(q, r, d, bits, page, R, W, codes, meta, K, V, n_valid, P, k, scale,
+                            0, page_idx, tok_idx, U, D, out, q_ambiguous);
 }
 
 }  // extern "C"

@@ -45,6 +45,12 @@ def lib():
             "hhro_attend": (None, [p, i32, i32, p, p, p, i64, f64, p]),
             "hhro_decode_unit": (i64, [p, i32, i32, i32, i32, p, p, p, p, p, p,
                                        i64, i64, i64, f64, p, p, p, p, p, p]),
+            "hhro_page_meta_f32": (None, [p, i64, i64, i32, i32, i64, i64, p]),
+            "hhro_encode_unit_f32": (i64, [p, i64, i64, i32, i32, i32, p, p, p, p]),
+            "hhro_page_bounds_f32": (None, [p, i32, i32, p, i64, p, p]),
+            "hhro_hamming_agg": (None, [p, i32, i32, p, p, i64, i32, i64, i32, p]),
+            "hhro_decode_unit_v": (i64, [p, i32, i32, i32, i32, p, p, p, p, p, p,
+                                         i64, i64, i64, f64, i32, p, p, p, p, p, p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -87,26 +93,29 @@ def project_sign(x_bits, W, want_z=False):
     return (codes, amb, z) if want_z else (codes, amb)
 
 
-def page_meta(kt, n_valid, page, p_begin=0, p_end=None, t0=0, meta=None):
-    """Extrema of §3.3.1 (Eq. 3) rounded outward to bf16: [np][2][d] uint16."""
+def page_meta(kt, n_valid, page, p_begin=0, p_end=None, t0=0, meta=None, f32=False):
+    """Extrema of §3.3.1 (Eq. 3): rounded outward to bf16, [np][2][d] uint16;
+    with ``f32`` (variant V1) kept as float32, [np][2][d] float32."""
     kt = _c(kt, np.float32)
     d = kt.shape[1]
     if p_end is None:
         p_end = (n_valid + page - 1) // page
     if meta is None:
-        meta = np.zeros((p_end, 2, d), np.uint16)
-    lib().hhro_page_meta(_p(kt), t0, n_valid, d, page, p_begin, p_end, _p(meta))
+        meta = np.zeros((p_end, 2, d), np.float32 if f32 else np.uint16)
+    fn = lib().hhro_page_meta_f32 if meta.dtype == np.float32 else lib().hhro_page_meta
+    fn(_p(kt), t0, n_valid, d, page, p_begin, p_end, _p(meta))
     return meta
 
 
 def encode_unit(K_unit, n_begin, n_end, page, R_g, W_g, codes_unit, meta_unit):
-    """Encode keys [n_begin, n_end) of one unit in place; returns ambiguous count."""
+    """Encode keys [n_begin, n_end) of one unit in place; returns ambiguous count.
+    A float32 ``meta_unit`` selects the float32-metadata variant (V1)."""
     assert K_unit.flags.c_contiguous and codes_unit.flags.c_contiguous and meta_unit.flags.c_contiguous
     d = K_unit.shape[1]
     bits = W_g.shape[1]
-    return lib().hhro_encode_unit(_p(K_unit), n_begin, n_end, d, bits, page,
-                                  _p(_c(R_g, np.float32)), _p(_c(W_g, np.float32)),
-                                  _p(codes_unit), _p(meta_unit))
+    fn = lib().hhro_encode_unit_f32 if meta_unit.dtype == np.float32 else lib().hhro_encode_unit
+    return fn(_p(K_unit), n_begin, n_end, d, bits, page, _p(_c(R_g, np.float32)),
+              _p(_c(W_g, np.float32)), _p(codes_unit), _p(meta_unit))
 
 
 def query_prep(q_bits, R_g, W_g):
@@ -122,13 +131,16 @@ def query_prep(q_bits, R_g, W_g):
 
 
 def page_bounds(qt, meta_unit, n_pages, per_head=False):
-    """§3.3.1 Eq. 3, max over the group's heads: U [np] float64 (, Uh [r][np])."""
+    """§3.3.1 Eq. 3, max over the group's heads: U [np] float64 (, Uh [r][np]).
+    bf16 (uint16) or float32 (variant V1) metadata."""
     qt = _c(qt, np.float32)
-    meta = _c(meta_unit, np.uint16)
+    f32 = np.asarray(meta_unit).dtype == np.float32
+    meta = _c(meta_unit, np.float32 if f32 else np.uint16)
     r, d = qt.shape
     U = np.empty(n_pages, np.float64)
     Uh = np.empty((r, n_pages), np.float64) if per_head else None
-    lib().hhro_page_bounds(_p(qt), r, d, _p(meta), n_pages, _p(U), _p(Uh))
+    fn = lib().hhro_page_bounds_f32 if f32 else lib().hhro_page_bounds
+    fn(_p(qt), r, d, _p(meta), n_pages, _p(U), _p(Uh))
     return (U, Uh) if per_head else U
 
 
@@ -139,13 +151,15 @@ def top_largest(s, m):
     return out[:cnt]
 
 
-def hamming(qcode, codes_unit, pages, page, n_valid):
+def hamming(qcode, codes_unit, pages, page, n_valid, gqa_sum=False):
+    """§3.1 Eq. 2 over the group's heads: min (reading R4) or sum (variant V2)."""
     qc = _c(qcode, np.uint32)
     codes = _c(codes_unit, np.uint32)
     pages = _c(pages, np.int32)
     r, words = qc.shape
     D = np.empty(pages.shape[0] * page, np.int32)
-    lib().hhro_hamming(_p(qc), r, words, _p(codes), _p(pages), pages.shape[0], page, n_valid, _p(D))
+    lib().hhro_hamming_agg(_p(qc), r, words, _p(codes), _p(pages), pages.shape[0], page, n_valid,
+                           1 if gqa_sum else 0, _p(D))
     return D
 
 
@@ -168,8 +182,9 @@ def attend(q_bits, K_unit, V_unit, idx, scale):
 
 
 def decode_unit(q_bits, R_g, W_g, codes_unit, meta_unit, K_unit, V_unit, n_valid, page, P, k,
-                scale, attend_too=True):
-    """One decode step of one unit; returns a dict of numpy outputs."""
+                scale, attend_too=True, gqa_sum=False):
+    """One decode step of one unit; returns a dict of numpy outputs.  A float32
+    ``meta_unit`` selects variant V1, ``gqa_sum`` variant V2."""
     q = _c(q_bits, np.uint16)
     r, d = q.shape
     bits = W_g.shape[1]
@@ -180,11 +195,13 @@ def decode_unit(q_bits, R_g, W_g, codes_unit, meta_unit, K_unit, V_unit, n_valid
     D = np.empty(P * page, np.int32)
     out = np.empty((r, d), np.float32) if attend_too else None
     amb = C.c_int64(0)
-    n_sel = lib().hhro_decode_unit(
+    f32 = np.asarray(meta_unit).dtype == np.float32
+    flags = (1 if f32 else 0) | (2 if gqa_sum else 0)
+    n_sel = lib().hhro_decode_unit_v(
         _p(q), r, d, bits, page, _p(_c(R_g, np.float32)), _p(_c(W_g, np.float32)),
-        _p(_c(codes_unit, np.uint32)), _p(_c(meta_unit, np.uint16)),
+        _p(_c(codes_unit, np.uint32)), _p(_c(meta_unit, np.float32 if f32 else np.uint16)),
         _p(_c(K_unit, np.uint16)), _p(_c(V_unit, np.uint16)),
-        n_valid, P, k, float(scale), _p(page_idx), _p(tok_idx), _p(U), _p(D), _p(out),
+        n_valid, P, k, float(scale), flags, _p(page_idx), _p(tok_idx), _p(U), _p(D), _p(out),
         C.byref(amb))
     return dict(page_idx=page_idx, tok_idx=tok_idx, n_sel=int(n_sel), U=U, D=D, out=out,
                 q_ambiguous=int(amb.value))
@@ -200,18 +217,20 @@ def _units(w, units):
     return [(b, g) for b in range(w.B) for g in range(w.Hkv)] if units is None else list(units)
 
 
-def encode_all(inp, n_begin=0, n_end=None, codes=None, meta=None, units=None, threads=None):
+def encode_all(inp, n_begin=0, n_end=None, codes=None, meta=None, units=None, threads=None,
+               meta_f32=False):
     """Oracle key encoding of ``inp`` (a ``workloads.Inputs``) for [n_begin, n_end).
 
-    Returns (codes [B][Hkv][n_cap][w] uint32, meta [B][Hkv][NPcap][2][d] uint16,
-    ambiguous count).  ``units`` restricts the work to some (b, g) pairs.
+    Returns (codes [B][Hkv][n_cap][w] uint32, meta [B][Hkv][NPcap][2][d] uint16
+    -- float32 with ``meta_f32`` (variant V1) --, ambiguous count).  ``units``
+    restricts the work to some (b, g) pairs.
     """
     w = inp.w
     n_end = w.N if n_end is None else n_end
     if codes is None:
         codes = np.zeros((w.B, w.Hkv, w.n_cap, w.words), np.uint32)
     if meta is None:
-        meta = np.zeros((w.B, w.Hkv, w.np_cap, 2, w.d), np.uint16)
+        meta = np.zeros((w.B, w.Hkv, w.np_cap, 2, w.d), np.float32 if meta_f32 else np.uint16)
     us = _units(w, units)
 
     def one(bg):
@@ -225,7 +244,7 @@ def encode_all(inp, n_begin=0, n_end=None, codes=None, meta=None, units=None, th
 
 
 def decode_all(inp, codes, meta, step=0, P=None, k=None, scale=None, attend_too=True,
-               units=None, threads=None):
+               units=None, threads=None, gqa_sum=False):
     """Oracle decode step ``step`` over all (or the listed) units.
 
     Returns dict with page_idx [B][Hkv][P], tok_idx [B][Hkv][k], n_sel [B][Hkv],
@@ -251,7 +270,7 @@ def decode_all(inp, codes, meta, step=0, P=None, k=None, scale=None, attend_too=
         b, g = bg
         return bg, decode_unit(inp.q[step, b, g * r:(g + 1) * r], inp.R[g], inp.W[g],
                                codes[b, g], meta[b, g], inp.K[b, g], inp.V[b, g],
-                               n_valid, w.page, P, k, scale, attend_too)
+                               n_valid, w.page, P, k, scale, attend_too, gqa_sum)
 
     with ThreadPoolExecutor(threads or default_threads()) as ex:
         for (b, g), o in ex.map(one, us):

@@ -389,3 +389,142 @@ def test_decode_unit_composes_the_primitives():
     assert np.array_equal(res["U"][(0, 0)], U)
     # the planted keys (logit ~ 3 |q| sqrt(d)) are found
     assert set(inp.planted_pos[0, 0].tolist()) <= set(tok.tolist())
+
+
+# ------------------------------------------- variants: float32 metadata (V1)
+
+def test_f32_metadata_is_exact_extrema():
+    """Variant V1 keeps the per-dimension extrema of §3.3.1 (under Eq. 3) in
+    float32 unrounded: numpy's min / max over each page's valid rows."""
+    rng = np.random.default_rng(21)
+    kt = (rng.standard_normal((16 * 7 + 9, 128)) * 5).astype(np.float32)
+    n_valid = kt.shape[0] - 4
+    meta = O.page_meta(kt, n_valid, 16, f32=True)
+    assert meta.dtype == np.float32 and meta.shape == (8, 2, 128)
+    for p in range(8):
+        rows = kt[p * 16:min((p + 1) * 16, n_valid)]
+        assert np.array_equal(meta[p, 0], rows.min(0))
+        assert np.array_equal(meta[p, 1], rows.max(0))
+
+
+def test_bf16_metadata_is_the_outward_rounding_of_f32_metadata():
+    """The default bf16 bounds are the float32 bounds of V1 rounded outward:
+    lo_bf16 <= lo_f32 with no bf16 value in between (and the mirror for hi)."""
+    rng = np.random.default_rng(22)
+    kt = (rng.standard_normal((16 * 5, 128)) * 9).astype(np.float32)
+    m16 = O.page_meta(kt, kt.shape[0], 16)
+    m32 = O.page_meta(kt, kt.shape[0], 16, f32=True)
+    lo16, hi16 = bf16_bits_to_f32(m16[:, 0]), bf16_bits_to_f32(m16[:, 1])
+    assert np.all(lo16 <= m32[:, 0]) and np.all(hi16 >= m32[:, 1])
+    lo_next = bf16_bits_to_f32(_next_toward_zero_or_up(m16[:, 0].ravel(), up=True)).reshape(lo16.shape)
+    hi_prev = bf16_bits_to_f32(_next_toward_zero_or_up(m16[:, 1].ravel(), up=False)).reshape(hi16.shape)
+    assert np.all((lo16 == m32[:, 0]) | (lo_next > m32[:, 0]))
+    assert np.all((hi16 == m32[:, 1]) | (hi_prev < m32[:, 1]))
+
+
+def test_f32_bound_is_the_rotated_logit_for_single_token_pages():
+    """With one key per page and float32 metadata the box of Eq. 3 is the point
+    k~ itself, so U = q~ . k~ (numpy dot in float64 of the float32 values),
+    which equals q . k up to the float32 rounding of the rotation (Eq. 4).  The
+    bf16 bound (outward rounding) can only be larger."""
+    rng = np.random.default_rng(23)
+    R, _ = make_rw(get("tiny_4k"))
+    k = _rand_bits(rng, (48, 128), 2.0)
+    q = _rand_bits(rng, (2, 128))
+    kt, qt = O.rotate(k, R[0]), O.rotate(q, R[0])
+    meta32 = O.page_meta(kt, 48, 1, f32=True)
+    _, Uh = O.page_bounds(qt, meta32, 48, per_head=True)
+    np.testing.assert_allclose(Uh, qt.astype(np.float64) @ kt.astype(np.float64).T, rtol=1e-12, atol=1e-12)
+    exact = _f(q) @ _f(k).T
+    scale = np.linalg.norm(_f(q), axis=1)[:, None] * np.linalg.norm(_f(k), axis=1)[None]
+    assert np.all(np.abs(Uh - exact) <= 1e-4 * scale)
+    _, Uh16 = O.page_bounds(qt, O.page_meta(kt, 48, 1), 48, per_head=True)
+    assert np.all(Uh16 >= Uh)
+
+
+def test_f32_bound_validity_and_tightness_on_generated_keys():
+    """V1 bounds stay >= every logit of their page (§3.3.1) and are never above
+    the bf16 bounds of the same keys."""
+    w = scaled(get("llama8b_32k"), B=1, Hkv=2, Hq=8, N=2500, planted=8)
+    inp = make_inputs(w)
+    codes16, meta16, _ = O.encode_all(inp, threads=2)
+    codes32, meta32, _ = O.encode_all(inp, threads=2, meta_f32=True)
+    assert meta32.dtype == np.float32 and np.array_equal(codes16, codes32)
+    np_ = w.n_pages()
+    for g in range(w.Hkv):
+        q = inp.q[0, 0, g * w.r:(g + 1) * w.r]
+        qt, _, _ = O.query_prep(q, inp.R[g], inp.W[g])
+        _, Uh = O.page_bounds(qt, meta32[0, g], np_, per_head=True)
+        _, Uh16 = O.page_bounds(qt, meta16[0, g], np_, per_head=True)
+        logits = _f(q) @ _f(inp.K[0, g, :w.N]).T
+        qtd = qt.astype(np.float64)
+        mag = np.maximum(np.abs(meta32[0, g, :np_, 0]), np.abs(meta32[0, g, :np_, 1])).astype(np.float64)
+        eps = 1e-5 * (np.abs(qtd)[:, None, :] * mag[None]).sum(-1)
+        for p in range(np_):
+            assert np.all(Uh[:, p] >= logits[:, p * 16:min((p + 1) * 16, w.N)].max(1) - eps[:, p])
+        assert np.all(Uh <= Uh16 + 1e-9 * np.abs(Uh16))
+
+
+def test_f32_append_encoding_equals_one_shot_encoding():
+    w = scaled(get("tiny_4k"), N=200, planted=2)
+    inp = make_inputs(w)
+    c1 = np.zeros((w.n_cap, 4), np.uint32)
+    m1 = np.zeros((w.np_cap, 2, 128), np.float32)
+    O.encode_unit(inp.K[0, 0], 0, 200, 16, inp.R[0], inp.W[0], c1, m1)
+    c2, m2 = np.zeros_like(c1), np.zeros_like(m1)
+    for a, b in [(0, 17), (17, 18), (18, 150), (150, 200)]:
+        O.encode_unit(inp.K[0, 0], a, b, 16, inp.R[0], inp.W[0], c2, m2)
+    assert np.array_equal(c1, c2) and np.array_equal(m1, m2)
+
+
+# ------------------------------------------------ variants: GQA-sum (V2)
+
+def test_gqa_sum_distance_matches_summed_sign_closed_form():
+    """Eq. 2 summed over the r heads of a group: with ±1 signs,
+    sum_h popc(c_h xor c) = (r b - (sum_h s_h) . s) / 2 -- one dot product of
+    the summed query signs with the key signs (numpy)."""
+    rng = np.random.default_rng(24)
+    for r, bits in ((4, 128), (2, 256), (8, 128)):
+        words = bits // 32
+        codes = rng.integers(0, 2**32, size=(64, words), dtype=np.uint64).astype(np.uint32)
+        qc = rng.integers(0, 2**32, size=(r, words), dtype=np.uint64).astype(np.uint32)
+        pages = np.array([0, 3], np.int32)
+        D = O.hamming(qc, codes, pages, 16, 60, gqa_sum=True)
+        sq = 2 * np.unpackbits(qc.view(np.uint8), bitorder="little").reshape(r, bits).astype(np.int64) - 1
+        sk = 2 * np.unpackbits(codes.view(np.uint8), bitorder="little").reshape(64, bits).astype(np.int64) - 1
+        for slot, p in enumerate(pages):
+            for t in range(16):
+                n = p * 16 + t
+                want = -1 if n >= 60 else (r * bits - int(sq.sum(0) @ sk[n])) // 2
+                assert D[slot * 16 + t] == want
+
+
+def test_gqa_sum_and_min_agree_for_one_head_and_differ_for_groups():
+    rng = np.random.default_rng(25)
+    codes = rng.integers(0, 2**32, size=(32, 4), dtype=np.uint64).astype(np.uint32)
+    pages = np.array([0, 1], np.int32)
+    q1 = rng.integers(0, 2**32, size=(1, 4), dtype=np.uint64).astype(np.uint32)
+    assert np.array_equal(O.hamming(q1, codes, pages, 16, 32, gqa_sum=True),
+                          O.hamming(q1, codes, pages, 16, 32))
+    q4 = rng.integers(0, 2**32, size=(4, 4), dtype=np.uint64).astype(np.uint32)
+    s, m = O.hamming(q4, codes, pages, 16, 32, gqa_sum=True), O.hamming(q4, codes, pages, 16, 32)
+    assert np.all(s >= 4 * m) and np.all(s <= 4 * 128) and not np.array_equal(s, m)
+
+
+def test_decode_unit_variants_compose_the_primitives():
+    """The flags of one decode step route to the variant primitives: float32
+    bounds (V1) and summed distances (V2), the rest unchanged."""
+    w = scaled(get("llama8b_32k"), B=1, Hkv=1, Hq=4, N=1800, P=25, k=90, planted=4)
+    inp = make_inputs(w)
+    codes, meta32, _ = O.encode_all(inp, threads=1, meta_f32=True)
+    for gqa_sum in (False, True):
+        res = O.decode_all(inp, codes, meta32, threads=1, gqa_sum=gqa_sum)
+        qt, qc, _ = O.query_prep(inp.q[0, 0], inp.R[0], inp.W[0])
+        U = O.page_bounds(qt, meta32[0, 0], w.n_pages())
+        pages = O.top_largest(U, 25)
+        D = O.hamming(qc, codes[0, 0], pages, 16, w.N, gqa_sum=gqa_sum)
+        tok = O.top_tokens(D, pages, 16, 90)
+        assert res["page_idx"][0, 0].tolist() == pages.tolist()
+        assert res["tok_idx"][0, 0].tolist() == tok.tolist()
+        assert res["D"][0, 0, :25 * 16].tolist() == D.tolist()
+        assert np.array_equal(res["U"][(0, 0)], U)
