@@ -29,6 +29,11 @@
  *     ties to the lower token index.  Nothing else is forced in.
  *   - Attention uses the original keys (Eq. 4 leaves logits unchanged) and the
  *     scale the caller passes (usually 1/sqrt(d)).
+ *   Two of these readings have a variant, chosen per call by hhr_dims.flags:
+ *   - HHR_FLAG_META_F32: page metadata is float32, the extrema exactly as
+ *     computed from the float32 rotated keys (no rounding; twice the bytes).
+ *   - HHR_FLAG_GQA_SUM: a token's distance is the sum over the group's heads
+ *     of Eq. 2 (range 0 .. r*bits) instead of the min.
  *
  * Conventions common to every call
  *   Memory.  The caller owns every buffer.  Pointers documented as "device"
@@ -54,7 +59,7 @@
  *     K, V      bf16 [B][Hkv][n_cap][d]          keys / values (KV cache)
  *     codes     u32  [B][Hkv][n_cap][bits/32]    bit t of a key's code is bit
  *                                                t%32 of word t/32
- *     meta      bf16 [B][Hkv][ceil(n_cap/page)][2][d]
+ *     meta      bf16 [B][Hkv][ceil(n_cap/page)][2][d]  (f32 with HHR_FLAG_META_F32)
  *                    [p][0][j]: lower bound of dimension j over page p
  *                    [p][1][j]: upper bound of dimension j over page p
  *     R         f32  [Hkv][d][d]                 k~[j] = sum_i k[i] R[i][j]
@@ -93,6 +98,10 @@ typedef enum hhr_status {
 /* Largest number of pages per (sequence, KV head) a decode call accepts. */
 #define HHR_MAX_PAGES 16384
 
+/* hhr_dims.flags: variants of two readings (see the top of this file). */
+#define HHR_FLAG_META_F32 1  /* meta is f32, unrounded extrema               */
+#define HHR_FLAG_GQA_SUM 2   /* token distance = sum over the group's heads  */
+
 typedef struct hhr_dims {
   int32_t B;     /* sequences                                   */
   int32_t Hq;    /* query heads                                 */
@@ -101,6 +110,7 @@ typedef struct hhr_dims {
   int32_t bits;  /* code length b (128 or 256)                  */
   int32_t page;  /* tokens per page S                           */
   int32_t n_cap; /* KV-cache capacity per (sequence, KV head)   */
+  int32_t flags; /* 0, or HHR_FLAG_META_F32 | HHR_FLAG_GQA_SUM  */
 } hhr_dims;
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */

@@ -30,16 +30,21 @@ class HhrError(RuntimeError):
         self.status = status
 
 
+HHR_FLAG_META_F32 = 1   # page metadata in float32 (unrounded extrema)
+HHR_FLAG_GQA_SUM = 2    # token distance = sum over the group's heads
+
+
 class hhr_dims(C.Structure):
     _fields_ = [("B", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32), ("d", C.c_int32),
-                ("bits", C.c_int32), ("page", C.c_int32), ("n_cap", C.c_int32)]
+                ("bits", C.c_int32), ("page", C.c_int32), ("n_cap", C.c_int32),
+                ("flags", C.c_int32)]
 
     def __repr__(self):
         return "hhr_dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
-def make_dims(B, Hq, Hkv, d, bits, page, n_cap) -> hhr_dims:
-    return hhr_dims(B, Hq, Hkv, d, bits, page, n_cap)
+def make_dims(B, Hq, Hkv, d, bits, page, n_cap, flags=0) -> hhr_dims:
+    return hhr_dims(B, Hq, Hkv, d, bits, page, n_cap, flags)
 
 
 _lib = None

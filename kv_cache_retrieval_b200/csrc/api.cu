@@ -28,6 +28,7 @@ int32_t check_dims(const hhr_dims* d) {
   if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->d < 1 || d->bits < 1 || d->page < 1 || d->n_cap < 1)
     return HHR_ERR_INVALID_ARG;
   if (d->Hq % d->Hkv != 0) return HHR_ERR_INVALID_ARG;
+  if (d->flags & ~(HHR_FLAG_META_F32 | HHR_FLAG_GQA_SUM)) return HHR_ERR_INVALID_ARG;
   const int r = d->Hq / d->Hkv;
   if (d->d != kD) return HHR_ERR_UNSUPPORTED;
   if (d->bits != 128 && d->bits != 256) return HHR_ERR_UNSUPPORTED;
@@ -39,6 +40,8 @@ int32_t check_dims(const hhr_dims* d) {
 }
 
 int np_cap_of(const hhr_dims* d) { return (d->n_cap + d->page - 1) / d->page; }
+
+int hbins_of(const hhr_dims* d) { return hist_bins(d->Hq / d->Hkv, d->bits, d->flags); }
 
 struct DeviceInfo {
   int sms = 0;
@@ -82,6 +85,7 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   if (int32_t st = device_info(&info)) return st;
   const int r = d->Hq / d->Hkv;
   const int units = d->B * d->Hkv;
+  const int hbins = hbins_of(d);
   const int NP = (n_valid + d->page - 1) / d->page;
   const int Pk = P < NP ? P : NP;
   // one CTA per SM (512 threads, up to 128 registers each)
@@ -95,6 +99,11 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   } else {
     const int by_pages = (NP + kMinPagesPerCta - 1) / kMinPagesPerCta;
     if (C > by_pages) C = by_pages < 1 ? 1 : by_pages;
+    // the unit's C distance histograms, their row prefixes and the totals
+    // share the scratch area with the metadata ring (192 KiB): with the wide
+    // GQA-sum histograms that caps C
+    const int by_hist = static_cast<int>((size_t{192} * 1024 / sizeof(int) - hbins - 4) / (2 * hbins + 1));
+    if (C > by_hist) C = by_hist < 1 ? 1 : by_hist;
   }
   int slice_pages = 0, slice_tokens = 0;
   for (;;) {
@@ -109,7 +118,7 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
     ++C;
   }
   if (slice_tokens > kMaxTokensPerCta) return HHR_ERR_UNSUPPORTED;
-  const DecodeSmem lay = decode_smem(NP, C, d->bits, r, slice_pages, slice_tokens, mode);
+  const DecodeSmem lay = decode_smem(NP, C, d->bits, r, slice_pages, slice_tokens, mode, hbins);
   if (lay.total > info.smem_optin) return HHR_ERR_UNSUPPORTED;
   int grid_units = resident / C;
   if (grid_units > units) grid_units = units;
@@ -132,12 +141,15 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   a->slice_pages = slice_pages;
   a->slice_tokens = slice_tokens;
   a->spin_limit = kSpinLimit;
+  a->meta_f32 = (d->flags & HHR_FLAG_META_F32) ? 1 : 0;
+  a->gqa_sum = (d->flags & HHR_FLAG_GQA_SUM) ? 1 : 0;
+  a->hbins = hbins;
   *smem = lay.total;
   return HHR_OK;
 }
 
 void carve_workspace(void* ws, const hhr_dims* d, DecodeArgs* a) {
-  const WsLayout L = ws_layout(d->B * d->Hkv, np_cap_of(d), d->Hq / d->Hkv, d->bits);
+  const WsLayout L = ws_layout(d->B * d->Hkv, np_cap_of(d), d->Hq / d->Hkv, hbins_of(d));
   unsigned char* base = static_cast<unsigned char*>(ws);
   a->status = reinterpret_cast<uint32_t*>(base + L.status);
   a->counters = reinterpret_cast<uint32_t*>(base + L.counters);
@@ -151,7 +163,7 @@ void carve_workspace(void* ws, const hhr_dims* d, DecodeArgs* a) {
 int32_t check_workspace(const hhr_dims* d, void* ws, size_t ws_bytes) {
   if (!ws) return HHR_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return HHR_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(d->B * d->Hkv, np_cap_of(d), d->Hq / d->Hkv, d->bits);
+  const WsLayout L = ws_layout(d->B * d->Hkv, np_cap_of(d), d->Hq / d->Hkv, hbins_of(d));
   if (ws_bytes < L.total) return HHR_ERR_WORKSPACE;
   return HHR_OK;
 }
@@ -204,7 +216,8 @@ int32_t hhr_encode_keys(const hhr_dims* dims, const void* K, const float* R, con
   a.R = R;
   a.W = W;
   a.codes = codes;
-  a.meta = static_cast<uint16_t*>(meta);
+  a.meta = meta;
+  a.meta_f32 = (dims->flags & HHR_FLAG_META_F32) ? 1 : 0;
   a.Hkv = dims->Hkv;
   a.units = dims->B * dims->Hkv;
   a.bits = dims->bits;
@@ -233,7 +246,7 @@ int32_t hhr_encode_keys(const hhr_dims* dims, const void* K, const float* R, con
 
 size_t hhr_workspace_size(const hhr_dims* dims, int32_t P, int32_t k) {
   if (check_dims(dims) != HHR_OK || P < 1 || k < 1) return 0;
-  const WsLayout L = ws_layout(dims->B * dims->Hkv, np_cap_of(dims), dims->Hq / dims->Hkv, dims->bits);
+  const WsLayout L = ws_layout(dims->B * dims->Hkv, np_cap_of(dims), dims->Hq / dims->Hkv, hbins_of(dims));
   return L.total;
 }
 
@@ -269,7 +282,7 @@ static int32_t decode_common(const hhr_dims* dims, int mode, const void* q, cons
   a.R = R;
   a.W = W;
   a.codes = codes;
-  a.meta = static_cast<const uint16_t*>(meta);
+  a.meta = meta;
   a.K = static_cast<const uint16_t*>(K);
   a.V = static_cast<const uint16_t*>(V);
   a.tok_in = tok_in;

@@ -362,6 +362,7 @@ __device__ __forceinline__ void put_terms(uint16_t* qb, int n0, int k, float v) 
 struct Smem {
   uint16_t* qb;    // bf16 terms of [min(q~, 0) ; max(q~, 0)], [8 nb][2 d], 16-B chunks swizzled
   float* qf;       // [r][d] queries (float), pre-scaled for attention
+  float* qt;       // [r][d] q~ = q R (float), for float32 metadata
   uint32_t* qc;    // [r][w] query codes
   int* my_pages;   // kept pages of this CTA's slice
   uint16_t* tokD;  // distances of the slice's tokens
@@ -677,10 +678,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
   constexpr int BITS = WORDS * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x % a.C;
-  const DecodeSmem lay = decode_smem(a.NP, a.C, BITS, RG, a.slice_pages, a.slice_tokens, MODE);
+  const DecodeSmem lay = decode_smem(a.NP, a.C, BITS, RG, a.slice_pages, a.slice_tokens, MODE, a.hbins);
   Smem S;
   S.qb = reinterpret_cast<uint16_t*>(smem + lay.qb);
   S.qf = reinterpret_cast<float*>(smem + lay.qf);
+  S.qt = reinterpret_cast<float*>(smem + lay.qt);
   S.qc = reinterpret_cast<uint32_t*>(smem + lay.qc);
   S.my_pages = reinterpret_cast<int*>(smem + lay.my_pages);
   S.tokD = reinterpret_cast<uint16_t*>(smem + lay.tokD);
@@ -785,19 +787,35 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       static_assert((kRingSlots - kLaneSlots) * NWARPS * 512 == kD * kD * sizeof(float),
                     "the upper ring slots fill the R / W buffer exactly");
       const int n_grp = (w_pages + PPG - 1) / PPG;
-      const uint16_t* meta_u = a.meta + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
-      const uint4* wsrc = reinterpret_cast<const uint4*>(meta_u + wpb * 2 * kD) + lane;  // 32 x 16 B per page
-      // Within a slot, 16-B chunk c sits at position c ^ (s & 7), so that the
-      // same chunk of 8 consecutive slots covers all banks (ldmatrix below).
+      // bf16 metadata: a page is 512 B (32 x 16 B), one slot.  Within a slot,
+      // 16-B chunk c sits at position c ^ (s & 7), so that the same chunk of 8
+      // consecutive slots covers all banks (ldmatrix below).
+      // f32 metadata: a page is 1 KiB, two slots (lower bounds, upper
+      // bounds), PPG / 2 pages per group; lane l keeps chunk l of each half at
+      // position l (it alone reads it back).
+      const size_t meta_row = static_cast<size_t>(unit) * a.np_cap + wpb;   // first page of the warp
+      const uint4* wsrc = reinterpret_cast<const uint4*>(a.meta) + meta_row * (a.meta_f32 ? 64 : 32) + lane;
       uint4* ring = reinterpret_cast<uint4*>(S.scratch) + warp * 32;
-      auto issue_group = [&](int gi) {  // every lane: its 16 B of PPG pages, one commit group
-        if (gi < n_grp) {
+      auto issue_group = [&](int gi) {  // every lane: its 16 B of each page half, one commit group
+        if (!a.meta_f32) {
+          if (gi < n_grp) {
 #pragma unroll
-          for (int pp = 0; pp < PPG; ++pp) {
-            const int pg = gi * PPG + pp;
-            const int s = pg % kRingSlots;
-            if (pg < w_pages)
-              cp_async16(ring + s * (NWARPS * 32) + (lane ^ (s & 7)), wsrc + static_cast<size_t>(pg) * 32);
+            for (int pp = 0; pp < PPG; ++pp) {
+              const int pg = gi * PPG + pp;
+              const int s = pg % kRingSlots;
+              if (pg < w_pages)
+                cp_async16(ring + s * (NWARPS * 32) + (lane ^ (s & 7)), wsrc + static_cast<size_t>(pg) * 32);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int pp = 0; pp < PPG / 2; ++pp) {
+            const int pg = gi * (PPG / 2) + pp;
+            const int s = (2 * pg) % kRingSlots;
+            if (pg < w_pages) {
+              cp_async16(ring + s * (NWARPS * 32) + lane, wsrc + static_cast<size_t>(pg) * 64);
+              cp_async16(ring + (s + 1) * (NWARPS * 32) + lane, wsrc + static_cast<size_t>(pg) * 64 + 32);
+            }
           }
         }
         cp_async_commit();
@@ -829,6 +847,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         for (int oi = tid; oi < RG * kD; oi += NT) {
           const float qt = product_sum<RG>(part, oi);
           const int h = oi / kD, j = oi % kD;
+          S.qt[oi] = qt;
           put_terms(S.qb, 4 * h, j, fminf(qt, 0.f));
           put_terms(S.qb, 4 * h, kD + j, fmaxf(qt, 0.f));
         }
@@ -852,66 +871,118 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       const int g8 = lane >> 2, t4 = lane & 3;      // mma fragment: row, column pair
       const uint32_t ring_s = smem_addr(S.scratch) + warp * 512;
       const uint32_t qb_s = smem_addr(S.qb);
-      for (int ti = 0; ti < n_tiles; ++ti) {
-        cp_async_wait<1>();   // this lane's groups 2 ti and 2 ti + 1 have landed
-        __syncwarp();         // ... and every lane's
-        // A row (lm & 1) * 8 + lr of the tile is page 16 ti + that row
-        const uint32_t a_row = ring_s + (((2 * ti + (lm & 1)) % GR) * PPG + lr) * (NWARPS * 512);
-        float acc[NB][4];
+      if (a.meta_f32) {
+        // Eq. 3 on float32 bounds, on the CUDA cores: lane l holds dimensions
+        // 4 l .. 4 l + 3 of a page's lower and upper bounds, forms
+        // sum_j min(q~_hj, 0) l_j + max(q~_hj, 0) u_j over them for every head,
+        // and the warp sums the 32 lanes (the path is bound by the 1-KiB pages'
+        // HBM traffic, not by this arithmetic).
+        float qv[RG][4];
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
+        for (int h = 0; h < RG; ++h) {
+          const float4 t = *reinterpret_cast<const float4*>(S.qt + h * kD + 4 * lane);
+          qv[h][0] = t.x;
+          qv[h][1] = t.y;
+          qv[h][2] = t.z;
+          qv[h][3] = t.w;
+        }
+        const int n_grp32 = (w_pages + PPG / 2 - 1) / (PPG / 2);
+        for (int gi = 0; gi < n_grp32; ++gi) {
+          cp_async_wait<GR - 1>();   // this lane's chunks of group gi have landed
+#pragma unroll 1
+          for (int pp = 0; pp < PPG / 2; ++pp) {
+            const int pl = gi * (PPG / 2) + pp;
+            if (pl >= w_pages) break;   // warp-uniform
+            const int sl = (2 * pl) % kRingSlots;
+            const float4 lo = *reinterpret_cast<const float4*>(ring + sl * (NWARPS * 32) + lane);
+            const float4 hi = *reinterpret_cast<const float4*>(ring + (sl + 1) * (NWARPS * 32) + lane);
+            float u = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nb][e] = 0.f;
-#pragma unroll 4
-        for (int ks = 0; ks < 2 * kD / 16; ++ks) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(a_row + (static_cast<uint32_t>((2 * ks + (lm >> 1)) ^ lr) << 4), a0, a1, a2, a3);
+            for (int h = 0; h < RG; ++h) {
+              float t = fminf(qv[h][0], 0.f) * lo.x;
+              t = fmaf(fmaxf(qv[h][0], 0.f), hi.x, t);
+              t = fmaf(fminf(qv[h][1], 0.f), lo.y, t);
+              t = fmaf(fmaxf(qv[h][1], 0.f), hi.y, t);
+              t = fmaf(fminf(qv[h][2], 0.f), lo.z, t);
+              t = fmaf(fmaxf(qv[h][2], 0.f), hi.z, t);
+              t = fmaf(fminf(qv[h][3], 0.f), lo.w, t);
+              t = fmaf(fmaxf(qv[h][3], 0.f), hi.w, t);
 #pragma unroll
-          for (int nb = 0; nb < NB; nb += 2) {
-            if (nb + 1 < NB) {
-              uint32_t b0, b1, b2, b3;
-              const int n = (nb + (lm >> 1)) * 8 + lr;
-              ldsm_x4(qb_s + n * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1, b2, b3);
-              mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
-              mma_bf16_16816(acc[nb + 1], a0, a1, a2, a3, b2, b3);
-            } else {
-              uint32_t b0, b1;
-              ldsm_x2(qb_s + (nb * 8 + lr) * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1);
-              mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
+              for (int o2 = 16; o2 >= 1; o2 >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o2);
+              u = fmaxf(u, t);
             }
-          }
-        }
-        __syncwarp();
-        issue_group(2 * ti + GR);       // refill the slots just read
-        issue_group(2 * ti + GR + 1);
-        // lane (g8, t4) holds columns 8 nb + 2 t4, + 1 (head 2 nb + t4 / 2)
-        // of tile rows g8 and g8 + 8: add the terms, then take the max over
-        // the heads
-        float u0 = -INFINITY, u1 = -INFINITY;
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          float s0 = acc[nb][0] + acc[nb][1];
-          float s1 = acc[nb][2] + acc[nb][3];
-          s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
-          s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
-          if (2 * nb + (t4 >> 1) >= RG) {
-            s0 = -INFINITY;
-            s1 = -INFINITY;
-          }
-          u0 = fmaxf(u0, fmaxf(s0, __shfl_xor_sync(0xFFFFFFFFu, s0, 2)));
-          u1 = fmaxf(u1, fmaxf(s1, __shfl_xor_sync(0xFFFFFFFFu, s1, 2)));
-        }
-        if (t4 == 0) {
-#pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            const int pl = ti * 16 + g8 + 8 * hr;
-            if (pl < w_pages) {
-              const float u = hr ? u1 : u0;
+            if (lane == 0) {
               const int pg = wpb + pl;
               wsU_u[pg] = u;
               if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
-              lmin = fminf(lmin, u);
-              lmax = fmaxf(lmax, u);
+            }
+            lmin = fminf(lmin, u);
+            lmax = fmaxf(lmax, u);
+          }
+          issue_group(gi + GR);   // refill this lane's slots of group gi
+        }
+      } else {
+        for (int ti = 0; ti < n_tiles; ++ti) {
+          cp_async_wait<1>();   // this lane's groups 2 ti and 2 ti + 1 have landed
+          __syncwarp();         // ... and every lane's
+          // A row (lm & 1) * 8 + lr of the tile is page 16 ti + that row
+          const uint32_t a_row = ring_s + (((2 * ti + (lm & 1)) % GR) * PPG + lr) * (NWARPS * 512);
+          float acc[NB][4];
+  #pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nb][e] = 0.f;
+  #pragma unroll 4
+          for (int ks = 0; ks < 2 * kD / 16; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(a_row + (static_cast<uint32_t>((2 * ks + (lm >> 1)) ^ lr) << 4), a0, a1, a2, a3);
+  #pragma unroll
+            for (int nb = 0; nb < NB; nb += 2) {
+              if (nb + 1 < NB) {
+                uint32_t b0, b1, b2, b3;
+                const int n = (nb + (lm >> 1)) * 8 + lr;
+                ldsm_x4(qb_s + n * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1, b2, b3);
+                mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
+                mma_bf16_16816(acc[nb + 1], a0, a1, a2, a3, b2, b3);
+              } else {
+                uint32_t b0, b1;
+                ldsm_x2(qb_s + (nb * 8 + lr) * 512 + (static_cast<uint32_t>((2 * ks + (lm & 1)) ^ lr) << 4), b0, b1);
+                mma_bf16_16816(acc[nb], a0, a1, a2, a3, b0, b1);
+              }
+            }
+          }
+          __syncwarp();
+          issue_group(2 * ti + GR);       // refill the slots just read
+          issue_group(2 * ti + GR + 1);
+          // lane (g8, t4) holds columns 8 nb + 2 t4, + 1 (head 2 nb + t4 / 2)
+          // of tile rows g8 and g8 + 8: add the terms, then take the max over
+          // the heads
+          float u0 = -INFINITY, u1 = -INFINITY;
+  #pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            float s0 = acc[nb][0] + acc[nb][1];
+            float s1 = acc[nb][2] + acc[nb][3];
+            s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
+            s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
+            if (2 * nb + (t4 >> 1) >= RG) {
+              s0 = -INFINITY;
+              s1 = -INFINITY;
+            }
+            u0 = fmaxf(u0, fmaxf(s0, __shfl_xor_sync(0xFFFFFFFFu, s0, 2)));
+            u1 = fmaxf(u1, fmaxf(s1, __shfl_xor_sync(0xFFFFFFFFu, s1, 2)));
+          }
+          if (t4 == 0) {
+  #pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+              const int pl = ti * 16 + g8 + 8 * hr;
+              if (pl < w_pages) {
+                const float u = hr ? u1 : u0;
+                const int pg = wpb + pl;
+                wsU_u[pg] = u;
+                if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
+                lmin = fminf(lmin, u);
+                lmax = fmaxf(lmax, u);
+              }
             }
           }
         }
@@ -1226,8 +1297,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // ---------------------------------------------------------- phase 4
       const int S_ = a.page;
       const int ntok = (ke - ks) * S_;
-      int* sHD = reinterpret_cast<int*>(S.scratch);  // [BITS + 1]
-      for (int i = tid; i <= BITS; i += NT) sHD[i] = 0;
+      const int HB = a.hbins;                          // distance bins: BITS + 1, or r BITS + 1 (GQA-sum)
+      int* sHD = reinterpret_cast<int*>(S.scratch);  // [HB]
+      for (int i = tid; i < HB; i += NT) sHD[i] = 0;
       uint32_t qc[RG][WORDS];
 #pragma unroll
       for (int h = 0; h < RG; ++h)
@@ -1255,15 +1327,16 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
               kc[w4 * 4 + 2] = t.z;
               kc[w4 * 4 + 3] = t.w;
             }
-            int best = 1 << 20;
+            int best = 1 << 20, total = 0;
 #pragma unroll
             for (int h = 0; h < RG; ++h) {
               int dist = 0;
 #pragma unroll
               for (int w = 0; w < WORDS; ++w) dist += __popc(qc[h][w] ^ kc[w]);
               best = min(best, dist);
+              total += dist;
             }
-            D = best;
+            D = a.gqa_sum ? total : best;   // Eq. 2 over the group: min, or sum (GQA-sum)
           }
           S.tokD[i] = static_cast<uint16_t>(D);
           if (dbgD) dbgD[static_cast<size_t>(ks + slot) * S_ + off] = (D == 0xFFFF) ? -1 : D;
@@ -1275,8 +1348,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         for (int i = Pk * S_ + tid; i < a.P * S_; i += NT) dbgD[i] = -1;
       __syncthreads();
       {
-        int32_t* hrow = a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * (BITS + 1);
-        for (int i = tid; i <= BITS; i += NT) hrow[i] = sHD[i];
+        int32_t* hrow = a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit + c) * HB;
+        for (int i = tid; i < HB; i += NT) hrow[i] = sHD[i];
       }
       // unit barrier 2 (the release by thread 0 covers the CTA's histogram
       // row through the CTA barrier)
@@ -1285,38 +1358,34 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       if (!unit_wait(ctr, 2u * static_cast<uint32_t>(a.C) + (a.test_extra_stage == 2 ? 1u : 0u), a, s_misc)) return;
 
       // ---------------------------------------------------------- phase 5
-      int* sHA = reinterpret_cast<int*>(S.scratch);  // [C][BITS + 1]
+      int* sHA = reinterpret_cast<int*>(S.scratch);  // [C][HB]
       {
         // one batch of 16-B copies (a plain load/store loop would wait out an
         // L2 round trip per element, the compiler cannot reorder the global
         // loads past the shared stores).  The unit's area holds
-        // kMaxCtasPerUnit rows of a multiple of 16 B, so rounding the copy up
-        // to whole chunks stays inside it.
-        const char* hall = reinterpret_cast<const char*>(a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit) * (BITS + 1));
-        const int chunks = (a.C * (BITS + 1) * 4 + 15) / 16;
+        // kMaxCtasPerUnit rows of HB ints, so rounding the copy up to whole
+        // 16-B chunks stays inside it.
+        const char* hall = reinterpret_cast<const char*>(a.wsHist + static_cast<size_t>(unit * kMaxCtasPerUnit) * HB);
+        const int chunks = (a.C * HB * 4 + 15) / 16;
         for (int i = tid; i < chunks; i += NT) cp_async16(reinterpret_cast<char*>(sHA) + 16 * i, hall + 16 * i);
         cp_async_commit();
         cp_async_wait<0>();
       }
       __syncthreads();
       // Every CTA row's exclusive prefix over the distances (warp per row:
-      // lane l owns bins [VPL l, VPL l + VPL), bin BITS + 1 empty, so that
-      // pre[cc][BITS + 1] is the row's total) and the unit totals tot[v]
-      // (thread v); then warp 0 alone finds the threshold distance T (the
-      // k_eff-th smallest), how many tokens at T are still needed, and each
-      // CTA's tie quota and output offset in CTA order.
-      constexpr int VPL = (BITS + 2 + 31) / 32;
-      int* sPre = sHA + a.C * (BITS + 1);                // [C][BITS + 2]
-      int* sTot = sPre + a.C * (BITS + 2);               // [BITS + 1]
+      // lane l owns bins [VPL l, VPL l + VPL), bin HB empty, so that
+      // pre[cc][HB] is the row's total) and the unit totals tot[v]; then
+      // warp 0 alone finds the threshold distance T (the k_eff-th smallest),
+      // how many tokens at T are still needed, and each CTA's tie quota and
+      // output offset in CTA order.
+      const int VPL = (HB + 1 + 31) / 32;
+      int* sPre = sHA + a.C * HB;                        // [C][HB + 1]
+      int* sTot = sPre + a.C * (HB + 1);                 // [HB]
       for (int cc = warp; cc < a.C; cc += NWARPS) {
-        const int* row = sHA + cc * (BITS + 1);
-        int hv[VPL], loc = 0;
-#pragma unroll
-        for (int e = 0; e < VPL; ++e) {
-          const int v = lane * VPL + e;
-          hv[e] = v <= BITS ? row[v] : 0;
-          loc += hv[e];
-        }
+        const int* row = sHA + cc * HB;
+        const int v0 = lane * VPL, v1 = min(v0 + VPL, HB);
+        int loc = 0;
+        for (int v = v0; v < v1; ++v) loc += row[v];
         int incl = loc;
 #pragma unroll
         for (int o2 = 1; o2 < 32; o2 <<= 1) {
@@ -1324,28 +1393,23 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           if (lane >= o2) incl += y;
         }
         int run = incl - loc;
-#pragma unroll
-        for (int e = 0; e < VPL; ++e) {
-          const int v = lane * VPL + e;
-          if (v <= BITS + 1) sPre[cc * (BITS + 2) + v] = run;
-          run += hv[e];
+        for (int v = v0; v < v1; ++v) {
+          sPre[cc * (HB + 1) + v] = run;
+          run += row[v];
         }
+        if (v0 <= HB && HB < v0 + VPL) sPre[cc * (HB + 1) + HB] = run;   // the row's total
       }
-      if (tid <= BITS) {
+      for (int v = tid; v < HB; v += NT) {
         int x = 0;
 #pragma unroll 6
-        for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * (BITS + 1) + tid];
-        sTot[tid] = x;
+        for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * HB + v];
+        sTot[v] = x;
       }
       __syncthreads();
       if (warp == 0) {
-        int xv[VPL], loc = 0;
-#pragma unroll
-        for (int e = 0; e < VPL; ++e) {
-          const int v = lane * VPL + e;
-          xv[e] = v <= BITS ? sTot[v] : 0;
-          loc += xv[e];
-        }
+        const int v0 = lane * VPL, v1 = min(v0 + VPL, HB);
+        int loc = 0;
+        for (int v = v0; v < v1; ++v) loc += sTot[v];
         int incl = loc;
 #pragma unroll
         for (int o2 = 1; o2 < 32; o2 <<= 1) {
@@ -1358,13 +1422,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         int T = -1, needT = 0;
         if (incl - loc < k_eff && incl >= k_eff) {
           int run = incl - loc;
-#pragma unroll
-          for (int e = 0; e < VPL; ++e) {
-            if (run < k_eff && run + xv[e] >= k_eff) {
-              T = lane * VPL + e;
+          for (int v = v0; v < v1; ++v) {
+            const int xv = sTot[v];
+            if (run < k_eff && run + xv >= k_eff) {
+              T = v;
               needT = k_eff - run;
             }
-            run += xv[e];
+            run += xv;
           }
         }
         const unsigned own = __ballot_sync(0xFFFFFFFFu, T >= 0);
@@ -1378,8 +1442,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           const int cc = c0 + lane;
           int below = 0, eq = 0;
           if (cc < a.C && T >= 0) {
-            below = sPre[cc * (BITS + 2) + T];
-            eq = sPre[cc * (BITS + 2) + T + 1] - below;
+            below = sPre[cc * (HB + 1) + T];
+            eq = sPre[cc * (HB + 1) + T + 1] - below;
           }
           int eq_in = eq;
 #pragma unroll

@@ -136,13 +136,36 @@ __device__ __forceinline__ void split3(float v, uint16_t& hi, uint16_t& mid, uin
   lo = __bfloat16_as_ushort(l);
 }
 
+// Stores the bounds of dimension j of one page at dst ([2][d]): bf16 rounded
+// outward (the default), or float32 as computed (HHR_FLAG_META_F32).  MERGE:
+// combined with the bounds already stored (keys encoded by an earlier call).
+template <bool MERGE>
+__device__ __forceinline__ void put_bounds(__nv_bfloat16* dst, int j, float mn, float mx) {
+  __nv_bfloat16 lo = __float2bfloat16_rd(mn), hi = __float2bfloat16_ru(mx);
+  if (MERGE) {
+    lo = __hmin(lo, dst[j]);
+    hi = __hmax(hi, dst[kD + j]);
+  }
+  dst[j] = lo;
+  dst[kD + j] = hi;
+}
+template <bool MERGE>
+__device__ __forceinline__ void put_bounds(float* dst, int j, float mn, float mx) {
+  if (MERGE) {
+    mn = fminf(mn, dst[j]);
+    mx = fmaxf(mx, dst[kD + j]);
+  }
+  dst[j] = mn;
+  dst[kD + j] = mx;
+}
+
 // Pages of S keys (a power of two, at most 64) over one chunk of 32 keys of a
 // tile whose keys are all new (no masking, no merge): tree reductions with
 // static register indices.  For S = 64 a page spans two chunks; its partial
 // extrema are carried in mn / mx.
-template <int S>
+template <int S, typename MT>
 __device__ __forceinline__ void full_chunk_extrema(const uint32_t (&v)[32], int ch, int key0,
-                                                   __nv_bfloat16* meta_u, int j, float& mn, float& mx) {
+                                                   MT* meta_u, int j, float& mn, float& mx) {
   constexpr int G = S < 32 ? S : 32;          // keys of one page inside this chunk
 #pragma unroll
   for (int p0 = 0; p0 < 32; p0 += G) {
@@ -167,19 +190,17 @@ __device__ __forceinline__ void full_chunk_extrema(const uint32_t (&v)[32], int 
       mx = -INFINITY;
     }
     const int first = key0 + ch * 32 + p0 - (S > 32 ? 32 : 0);
-    __nv_bfloat16* dstp = meta_u + static_cast<size_t>(first / S) * 2 * kD;
-    dstp[j] = __float2bfloat16_rd(pmn);
-    dstp[kD + j] = __float2bfloat16_ru(pmx);
+    put_bounds<false>(meta_u + static_cast<size_t>(first / S) * 2 * kD, j, pmn, pmx);
   }
 }
 
 // Running per-page extrema over 32 keys (columns ch * 32 .. + 31 of the
-// tile) of output dimension j; a page's bounds are rounded outward to bf16
-// and stored when its last key has been seen.  MERGE: pages that start below
-// n_begin are merged with the bounds already stored.
-template <bool MERGE>
+// tile) of output dimension j; a page's bounds are stored (put_bounds) when
+// its last key has been seen.  MERGE: pages that start below n_begin are
+// merged with the bounds already stored.
+template <bool MERGE, typename MT>
 __device__ __forceinline__ void page_extrema(const uint32_t (&v)[32], int ch, int key0, int S, int n_begin,
-                                             int n_end, __nv_bfloat16* meta_u, int j, float& mn, float& mx) {
+                                             int n_end, MT* meta_u, int j, float& mn, float& mx) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int col = ch * 32 + i, key = key0 + col;
@@ -191,14 +212,11 @@ __device__ __forceinline__ void page_extrema(const uint32_t (&v)[32], int ch, in
     if (((col + 1) & (S - 1)) == 0) {   // the page ends at this key
       if (mn <= mx) {
         const int first = key + 1 - S;
-        __nv_bfloat16 lo = __float2bfloat16_rd(mn), hi = __float2bfloat16_ru(mx);
-        __nv_bfloat16* dstp = meta_u + static_cast<size_t>(first / S) * 2 * kD;
-        if (MERGE && first < n_begin) {  // keys [first, n_begin) were encoded before
-          lo = __hmin(lo, dstp[j]);
-          hi = __hmax(hi, dstp[kD + j]);
-        }
-        dstp[j] = lo;
-        dstp[kD + j] = hi;
+        MT* dstp = meta_u + static_cast<size_t>(first / S) * 2 * kD;
+        if (MERGE && first < n_begin)    // keys [first, n_begin) were encoded before
+          put_bounds<true>(dstp, j, mn, mx);
+        else
+          put_bounds<false>(dstp, j, mn, mx);
       }
       mn = INFINITY;
       mx = -INFINITY;
@@ -344,7 +362,6 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a)
       const int key0 = a.tile_begin + (it % a.n_tiles) * kTileKeys;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * kAccCols;
       float mn = INFINITY, mx = -INFINITY;                  // running extrema of the current page
-      __nv_bfloat16* meta_u = reinterpret_cast<__nv_bfloat16*>(a.meta) + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
       uint32_t* codes_u = a.codes + static_cast<size_t>(unit) * a.n_cap * words;
 #pragma unroll 1
       for (int ch = 0; ch < kTileKeys / 32; ++ch) {
@@ -353,21 +370,28 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a)
         if (ob == 0) {
           // only a tile that starts below n_begin holds a page with keys
           // encoded by an earlier call (its bounds are merged, not replaced)
-          if (key0 >= a.n_begin && key0 + kTileKeys <= a.n_end) {
-            switch (S) {
-              case 1: full_chunk_extrema<1>(v, ch, key0, meta_u, j, mn, mx); break;
-              case 2: full_chunk_extrema<2>(v, ch, key0, meta_u, j, mn, mx); break;
-              case 4: full_chunk_extrema<4>(v, ch, key0, meta_u, j, mn, mx); break;
-              case 8: full_chunk_extrema<8>(v, ch, key0, meta_u, j, mn, mx); break;
-              case 16: full_chunk_extrema<16>(v, ch, key0, meta_u, j, mn, mx); break;
-              case 32: full_chunk_extrema<32>(v, ch, key0, meta_u, j, mn, mx); break;
-              default: full_chunk_extrema<64>(v, ch, key0, meta_u, j, mn, mx); break;
+          auto extrema = [&](auto* meta_base) {
+            auto* meta_u = meta_base + static_cast<size_t>(unit) * a.np_cap * 2 * kD;
+            if (key0 >= a.n_begin && key0 + kTileKeys <= a.n_end) {
+              switch (S) {
+                case 1: full_chunk_extrema<1>(v, ch, key0, meta_u, j, mn, mx); break;
+                case 2: full_chunk_extrema<2>(v, ch, key0, meta_u, j, mn, mx); break;
+                case 4: full_chunk_extrema<4>(v, ch, key0, meta_u, j, mn, mx); break;
+                case 8: full_chunk_extrema<8>(v, ch, key0, meta_u, j, mn, mx); break;
+                case 16: full_chunk_extrema<16>(v, ch, key0, meta_u, j, mn, mx); break;
+                case 32: full_chunk_extrema<32>(v, ch, key0, meta_u, j, mn, mx); break;
+                default: full_chunk_extrema<64>(v, ch, key0, meta_u, j, mn, mx); break;
+              }
+            } else if (key0 < a.n_begin) {
+              page_extrema<true>(v, ch, key0, S, a.n_begin, a.n_end, meta_u, j, mn, mx);
+            } else {
+              page_extrema<false>(v, ch, key0, S, a.n_begin, a.n_end, meta_u, j, mn, mx);
             }
-          } else if (key0 < a.n_begin) {
-            page_extrema<true>(v, ch, key0, S, a.n_begin, a.n_end, meta_u, j, mn, mx);
-          } else {
-            page_extrema<false>(v, ch, key0, S, a.n_begin, a.n_end, meta_u, j, mn, mx);
-          }
+          };
+          if (a.meta_f32)
+            extrema(static_cast<float*>(a.meta));
+          else
+            extrema(static_cast<__nv_bfloat16*>(a.meta));
         } else {
           uint32_t mine = 0u;
 #pragma unroll

@@ -29,13 +29,19 @@ inline __host__ __device__ size_t align_up(size_t x, size_t a) { return (x + a -
 // padded to a multiple of four so it can be moved with 16-B accesses.
 inline __host__ __device__ constexpr int part_stride(int r) { return (r * (kD + 2) + 3) / 4 * 4; }
 
+// Bins of a token-distance histogram: distances 0 .. bits (min over the
+// group's heads) or 0 .. r * bits (HHR_FLAG_GQA_SUM).
+inline __host__ __device__ int hist_bins(int r, int bits, int flags) {
+  return ((flags & HHR_FLAG_GQA_SUM) ? r * bits : bits) + 1;
+}
+
 // Workspace layout (bytes).  The status word sits at offset 0.
 struct WsLayout {
   size_t status, counters, U, minmax, hist, part, total;
   int np_stride;  // floats per unit in the U area (multiple of 4)
 };
 
-inline __host__ __device__ WsLayout ws_layout(int units, int np_cap, int r, int bits) {
+inline __host__ __device__ WsLayout ws_layout(int units, int np_cap, int r, int hbins) {
   WsLayout L;
   size_t off = 0;
   L.status = off;   off += 256;
@@ -43,7 +49,7 @@ inline __host__ __device__ WsLayout ws_layout(int units, int np_cap, int r, int 
   L.np_stride = (int)align_up((size_t)np_cap, 4);
   L.U = off;        off += align_up(sizeof(float) * (size_t)units * L.np_stride, 256);
   L.minmax = off;   off += align_up(sizeof(float) * 2 * (size_t)units * kMaxCtasPerUnit, 256);
-  L.hist = off;     off += align_up(sizeof(int32_t) * (size_t)units * kMaxCtasPerUnit * (bits + 1), 256);
+  L.hist = off;     off += align_up(sizeof(int32_t) * (size_t)units * kMaxCtasPerUnit * hbins, 256);
   L.part = off;     off += align_up(sizeof(float) * (size_t)units * kMaxCtasPerUnit * part_stride(r), 256);
   L.total = off;
   return L;
@@ -57,7 +63,7 @@ struct DecodeArgs {
   const float* R;           // [Hkv][d][d]
   const float* W;           // [Hkv][d][bits]
   const uint32_t* codes;    // [B][Hkv][n_cap][w]
-  const uint16_t* meta;     // bf16 [B][Hkv][np_cap][2][d]
+  const void* meta;         // bf16 (f32 if meta_f32) [B][Hkv][np_cap][2][d]
   const uint16_t* K;        // bf16 [B][Hkv][n_cap][d]
   const uint16_t* V;
   const int32_t* tok_in;    // attend-only: [B][Hkv][k]
@@ -84,6 +90,9 @@ struct DecodeArgs {
   float scale_log2;         // scale * log2(e)
   unsigned long long spin_limit;
   int test_extra_stage;     // test hook: unit barrier (1 or 2) that waits for one arrival too many; 0 = none
+  int meta_f32;             // HHR_FLAG_META_F32: f32 metadata, bounds by SIMT
+  int gqa_sum;              // HHR_FLAG_GQA_SUM: distance = sum over the group's heads
+  int hbins;                // distance histogram bins (hist_bins)
 };
 
 struct EncodeArgs {
@@ -91,18 +100,19 @@ struct EncodeArgs {
   const float* R;
   const float* W;
   uint32_t* codes;
-  uint16_t* meta;
+  void* meta;                      // bf16, or f32 when meta_f32
   int Hkv, units, bits, page, n_cap, np_cap, n_begin, n_end, tile_begin, n_tiles;
+  int meta_f32;                    // HHR_FLAG_META_F32: unrounded f32 extrema
   unsigned long long spin_limit;   // clock cycles a pipeline wait may take
   int test_extra_arrival;          // test hook: the first stage waits for one producer arrival too many
 };
 
 // Shared-memory bytes of a decode CTA (host and device agree on the carve-up).
 struct DecodeSmem {
-  size_t qb, qf, qc, my_pages, tokD, sel, scratch, total;
+  size_t qb, qf, qt, qc, my_pages, tokD, sel, scratch, total;
 };
 
-inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, int r, int mode) {
+inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int r, int mode, int hbins) {
   size_t sel = 0, hist = 0, attn = 0, stream = 0;
   if (mode != kModeAttend) {
     // per-warp metadata rings; their upper slots double as R / W staging
@@ -113,7 +123,7 @@ inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, 
         + 2 * (sizeof(float) + sizeof(int)) * kCandMax       // boundary candidates, 2 levels
         + sizeof(float) * 2 * (kDecodeThreads / 32);          // level-2 min / max
     // distance histograms, their row prefixes, the unit totals (+ copy rounding)
-    hist = sizeof(int) * ((size_t)C * (bits + 1) + (size_t)C * (bits + 2) + (bits + 1)) + 16;
+    hist = sizeof(int) * ((size_t)C * hbins + (size_t)C * (hbins + 1) + hbins) + 16;
   }
   if (mode != kModeSelect) {
     // per warp: K and V of 16 tokens; then the 16-row query tile
@@ -127,16 +137,17 @@ inline __host__ __device__ size_t decode_scratch_bytes(int NP, int C, int bits, 
 }
 
 inline __host__ __device__ DecodeSmem decode_smem(int NP, int C, int bits, int r, int slice_pages,
-                                                  int slice_tokens, int mode) {
+                                                  int slice_tokens, int mode, int hbins) {
   DecodeSmem s;
   size_t off = 0;
   s.qb = off;       off += (size_t)8 * ((r * 4 + 7) / 8) * 2 * kD * 2;  // bf16 terms of q~, [8 nb][2 d]
   s.qf = off;       off += align_up(sizeof(float) * r * kD, 16);
+  s.qt = off;       off += align_up(sizeof(float) * r * kD, 16);          // q~ (f32-metadata bounds)
   s.qc = off;       off += align_up(sizeof(uint32_t) * r * (bits / 32), 16);
   s.my_pages = off; off += align_up(sizeof(int) * (size_t)(slice_pages + 1), 16);
   s.tokD = off;     off += align_up(sizeof(uint16_t) * (size_t)(slice_tokens + 1), 16);
   s.sel = off;      off += align_up(sizeof(int) * (size_t)(slice_tokens + 1), 16);
-  s.scratch = off;  off += align_up(decode_scratch_bytes(NP, C, bits, r, mode), 16);
+  s.scratch = off;  off += align_up(decode_scratch_bytes(NP, C, r, mode, hbins), 16);
   s.total = off;
   return s;
 }

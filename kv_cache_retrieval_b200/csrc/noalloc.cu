@@ -61,7 +61,7 @@ extern "C" int32_t hhr_decode_step_noalloc(const hhr_dims* dims, const void* q, 
   // reads it.  The rest of the scratch is written before it is read.
   const hhr::WsLayout L =
       hhr::ws_layout(dims->B * dims->Hkv, (dims->n_cap + dims->page - 1) / dims->page,
-                     dims->Hq / dims->Hkv, dims->bits);
+                     dims->Hq / dims->Hkv, hhr::hist_bins(dims->Hq / dims->Hkv, dims->bits, dims->flags));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + L.counters, 0, L.U - L.counters, s) != cudaSuccess)
     return HHR_ERR_CUDA;

@@ -42,20 +42,22 @@ def u32_host(t: torch.Tensor) -> np.ndarray:
 class Dev:
     """Device copies of a workload's inputs plus output buffers."""
 
-    def __init__(self, inp, P=None, k=None):
+    def __init__(self, inp, P=None, k=None, flags=0):
         w = inp.w
         self.w = w
         self.inp = inp
         self.P = w.P if P is None else P
         self.k = w.k if k is None else k
-        self.dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap)
+        self.flags = flags
+        self.dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap, flags)
         self.K = bf16_dev(inp.K)
         self.V = bf16_dev(inp.V)
         self.q = bf16_dev(inp.q)                   # [steps][B][Hq][d]
         self.R = torch.from_numpy(inp.R).cuda()
         self.W = torch.from_numpy(inp.W).cuda()
         self.codes = torch.zeros(w.B, w.Hkv, w.n_cap, w.words, dtype=torch.int32, device="cuda")
-        self.meta = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=torch.bfloat16, device="cuda")
+        meta_dtype = torch.float32 if flags & hhr.HHR_FLAG_META_F32 else torch.bfloat16
+        self.meta = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=meta_dtype, device="cuda")
         self.page_idx = torch.full((w.B, w.Hkv, self.P), -7, dtype=torch.int32, device="cuda")
         self.tok_idx = torch.full((w.B, w.Hkv, self.k), -7, dtype=torch.int32, device="cuda")
         self.n_sel = torch.full((w.B, w.Hkv), -7, dtype=torch.int32, device="cuda")
@@ -71,7 +73,14 @@ class Dev:
     def load_state(self, codes: np.ndarray, meta: np.ndarray):
         """Use oracle-encoded codes / metadata (identical bytes) as the state."""
         self.codes.copy_(u32_dev(codes))
-        self.meta.copy_(bf16_dev(meta))
+        if meta.dtype == np.float32:
+            self.meta.copy_(torch.from_numpy(np.ascontiguousarray(meta)).cuda())
+        else:
+            self.meta.copy_(bf16_dev(meta))
+
+    def meta_host(self) -> np.ndarray:
+        """The metadata as the oracle stores it: bf16 bits, or float32."""
+        return self.meta.cpu().numpy() if self.meta.dtype == torch.float32 else bits_host(self.meta)
 
     def select(self, step=0, n_valid=None, dbg=True):
         w = self.w
@@ -100,10 +109,12 @@ class Dev:
 
 def compare_encode(inp, codes_g, meta_g, units, n_end, n_begin=0):
     """Codes bit-exact except oracle |z| < 1e-4; metadata equal (a differing
-    bound may only be one bf16 step further out or in, reported)."""
+    bound may only be one bf16 step further out or in, reported).  float32
+    metadata (meta_g float32): equal up to the float32 rotation error."""
     w = inp.w
+    f32 = meta_g.dtype == np.float32
     report = dict(code_bits=0, ambiguous=0, meta_vals=0, meta_diff=0)
-    codes_o, meta_o, _ = O.encode_all(inp, n_begin=0, n_end=n_end, units=units)
+    codes_o, meta_o, _ = O.encode_all(inp, n_begin=0, n_end=n_end, units=units, meta_f32=f32)
     for (b, g) in units:
         c_o, _, z = O.project_sign(inp.K[b, g, n_begin:n_end], inp.W[g], want_z=True)
         c_g = codes_g[b, g, n_begin:n_end]
@@ -115,8 +126,8 @@ def compare_encode(inp, codes_g, meta_g, units, n_end, n_begin=0):
         report["code_bits"] += bits_o.size
         report["ambiguous"] += int(amb.sum())
         p0, p1 = n_begin // w.page, (n_end + w.page - 1) // w.page
-        mo = meta_o[b, g, p0:p1].astype(np.int32)
-        mg = meta_g[b, g, p0:p1].astype(np.int32)
+        mo = meta_o[b, g, p0:p1] if f32 else meta_o[b, g, p0:p1].astype(np.int32)
+        mg = meta_g[b, g, p0:p1] if f32 else meta_g[b, g, p0:p1].astype(np.int32)
         diff = mo != mg
         report["meta_vals"] += mo.size
         report["meta_diff"] += int(diff.sum())
@@ -131,9 +142,13 @@ def compare_encode(inp, codes_g, meta_g, units, n_end, n_begin=0):
             pad = (p1 - p0) * w.page - mag.shape[0]
             mag = np.pad(mag, ((0, pad), (0, 0))).reshape(p1 - p0, w.page, w.d).max(1)
             eps = np.broadcast_to((1e-5 * mag)[:, None, :], mo.shape)
-            fo = bf16_bits_to_f32(meta_o[b, g, p0:p1]).astype(np.float64)
-            fg = bf16_bits_to_f32(meta_g[b, g, p0:p1]).astype(np.float64)
-            step = np.maximum(np.abs(fo), np.abs(fg)) * 2.0 ** -7
+            if f32:
+                fo, fg = mo.astype(np.float64), mg.astype(np.float64)
+                step = 0.0
+            else:
+                fo = bf16_bits_to_f32(meta_o[b, g, p0:p1]).astype(np.float64)
+                fg = bf16_bits_to_f32(meta_g[b, g, p0:p1]).astype(np.float64)
+                step = np.maximum(np.abs(fo), np.abs(fg)) * 2.0 ** -7
             ok = np.abs(fo - fg) <= eps + step + 1e-30
             assert np.all(ok[diff]), "metadata differs by more than the float32 rotation error"
     return report

@@ -145,6 +145,70 @@ def test_rope_appends_each_step():
     assert d.status() == hhr.HHR_OK
 
 
+# ------------------------------------------------------------------ variants
+
+VARIANTS = {
+    "meta_f32": hhr.HHR_FLAG_META_F32,
+    "gqa_sum": hhr.HHR_FLAG_GQA_SUM,
+    "both": hhr.HHR_FLAG_META_F32 | hhr.HHR_FLAG_GQA_SUM,
+}
+_vcache = {}
+
+
+def variant_state(name, f32):
+    """Oracle-encoded codes and metadata of a small case (float32 metadata
+    with f32)."""
+    key = (name, f32)
+    if key not in _vcache:
+        inp, _, _ = case(name)
+        codes, meta, _ = O.encode_all(inp, n_end=inp.w.N, meta_f32=f32)
+        _vcache[key] = (codes, meta)
+    return _vcache[key]
+
+
+@pytest.mark.parametrize("variant", list(VARIANTS))
+@pytest.mark.parametrize("name", ["llama_20k_ragged", "b256_s32", "gqa8", "page1", "tiny_4k"])
+def test_variant_matches_oracle(name, variant):
+    """HHR_FLAG_META_F32 (float32 page metadata) and HHR_FLAG_GQA_SUM (summed
+    group distances) against the oracle's variants: the GPU encode, the
+    selection with its debug bounds / distances on the oracle's state, and
+    the fused step on the GPU-encoded state."""
+    inp, _, _ = case(name)
+    w = inp.w
+    flags = VARIANTS[variant]
+    f32 = bool(flags & hhr.HHR_FLAG_META_F32)
+    gsum = bool(flags & hhr.HHR_FLAG_GQA_SUM)
+    codes, meta = variant_state(name, f32)
+    d = Dev(inp, flags=flags)
+    d.encode(0, w.N)
+    torch.cuda.synchronize()
+    compare_encode(inp, u32_host(d.codes), d.meta_host(), all_units(w), w.N)
+    ores = O.decode_all(inp, codes, meta, gqa_sum=gsum)
+    s = Dev(inp, flags=flags)
+    s.load_state(codes, meta)
+    s.select(step=0)
+    assert s.status() == hhr.HHR_OK
+    compare_select(w, ores, _host(s.page_idx), _host(s.tok_idx), _host(s.n_sel), all_units(w),
+                   dbg_U=_host(s.dbg_U), dbg_D=_host(s.dbg_D), name=f"select {variant} {name}")
+    d.decode(0)
+    assert d.status() == hhr.HHR_OK
+    compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), all_units(w),
+                   inp=inp, step=0, out_g=_host(d.out), name=f"fused {variant} {name}")
+
+
+def test_variant_flags_are_validated():
+    inp, _, _ = case("tiny_4k")
+    w = inp.w
+    d = Dev(inp)
+    bad = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap, 4)
+    with pytest.raises(hhr.HhrError) as e:
+        hhr.hhr_encode_keys(bad, d.K, d.R, d.W, 0, w.N, d.codes, d.meta)
+    assert e.value.status == hhr.HHR_ERR_INVALID_ARG
+    # the summed distances need wider histograms: a larger workspace
+    sumd = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap, hhr.HHR_FLAG_GQA_SUM)
+    assert hhr.hhr_workspace_size(sumd, w.P, w.k) >= hhr.hhr_workspace_size(d.dims, w.P, w.k)
+
+
 # ------------------------------------------------------------------ edge cases
 
 @pytest.mark.parametrize("n_valid", [0, 1, 5, 16, 17, 333, 4096])
@@ -293,6 +357,7 @@ FULL_SAMPLES = {
     "llama8b_128k": [(0, 3), (0, 7)],
     "batch8_64k_b256": [(0, 0), (5, 2), (7, 7)],
     "qwen8b_128k_rope": [(1, 4), (3, 0)],
+    "llama8b_128k_paper": [(0, 1), (0, 6)],
 }
 
 
@@ -329,3 +394,26 @@ def test_full_size_sampled_units(name):
     torch.cuda.synchronize()
     rep = compare_encode(inp, u32_host(d.codes), bits_host(d.meta), units, inp.n_valid(steps[-1]))
     print(name, rep)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("variant", ["meta_f32", "gqa_sum"])
+def test_full_size_variants_sampled_units(variant):
+    """The variants at 128K in the launch configuration the benchmark times,
+    on sampled units (GPU encode, fused step)."""
+    w = get("llama8b_128k")
+    inp = make_inputs(w)
+    units = [(0, 2), (0, 5)]
+    flags = VARIANTS[variant]
+    f32 = bool(flags & hhr.HHR_FLAG_META_F32)
+    d = Dev(inp, flags=flags)
+    d.encode(0, w.N)
+    d.decode(0)
+    codes, meta, _ = O.encode_all(inp, 0, w.N, units=units, meta_f32=f32)
+    ores = O.decode_all(inp, codes, meta, units=units, gqa_sum=bool(flags & hhr.HHR_FLAG_GQA_SUM))
+    rep = compare_select(w, ores, _host(d.page_idx), _host(d.tok_idx), _host(d.n_sel), units,
+                         inp=inp, step=0, out_g=_host(d.out), name=f"full {variant} llama8b_128k")
+    print(variant, rep)
+    assert d.status() == hhr.HHR_OK
+    torch.cuda.synchronize()
+    compare_encode(inp, u32_host(d.codes), d.meta_host(), units, w.N)

@@ -1,4 +1,4 @@
-"""The five synthetic decode workloads that parity tests and the benchmark run.
+"""The synthetic decode workloads that parity tests and the benchmark run.
 
 Shapes follow the long-context decode settings of "HHR: Hierarchical Hash
 Retrieval for Efficient LLM Generation" (arXiv 2610.01230): Llama-3.1-8B /
@@ -80,6 +80,12 @@ WORKLOADS = {
         k=2048, bits=256, planted=64, n_outlier=round(0.05 * 128),
         outlier_scale=10.0, seed=_SEED0 + 3,
         notes="batched long-context decode, 256-bit codes, 32-token pages"),
+    "llama8b_128k_paper": Workload(
+        name="llama8b_128k_paper", B=1, Hq=32, Hkv=8, d=128, N=131072, page=16, P=2458,
+        k=1966, bits=128, planted=64, n_outlier=4, outlier_scale=8.0,
+        seed=_SEED0 + 2,
+        notes="the 128K inputs with the paper's ratios: candidate budget 30% of the "
+              "pages, Top-K 1.5% of the keys (Appendix A; §4.1)"),
     "qwen8b_128k_rope": Workload(
         name="qwen8b_128k_rope", B=4, Hq=32, Hkv=8, d=128, N=131072, page=16,
         P=512, k=4096, bits=128, planted=128, n_outlier=4, outlier_scale=8.0,
@@ -88,7 +94,8 @@ WORKLOADS = {
 }
 
 # Order used by tests and docs: the tiny case first, the headline case third.
-ORDER = ["tiny_4k", "llama8b_32k", "llama8b_128k", "batch8_64k_b256", "qwen8b_128k_rope"]
+ORDER = ["tiny_4k", "llama8b_32k", "llama8b_128k", "batch8_64k_b256", "qwen8b_128k_rope",
+         "llama8b_128k_paper"]
 
 HEADLINE = "llama8b_128k"
 
