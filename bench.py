@@ -71,15 +71,16 @@ def host_info():
     return model, os.cpu_count()
 
 
-def algorithmic_bytes(w, n_valid, P, k):
-    """Bytes a decode step must move at least once (read or write)."""
+def algorithmic_bytes(w, n_valid, P, k, meta_bytes=2):
+    """Bytes a decode step must move at least once (read or write);
+    meta_bytes = 4 for float32 page metadata."""
     units = w.B * w.Hkv
     NP = (n_valid + w.page - 1) // w.page
     Pk = min(P, NP)
     cand = min(Pk * w.page, n_valid)
     kk = min(k, cand)
     parts = dict(
-        meta=units * NP * 2 * w.d * 2,            # bf16 lower/upper bounds of every page
+        meta=units * NP * 2 * w.d * meta_bytes,   # lower/upper bounds of every page
         codes=units * cand * w.bits // 8,         # codes of the kept pages' tokens
         kv=units * kk * 2 * w.d * 2,              # gathered K and V rows
         rw=w.Hkv * (w.d * w.d + w.d * w.bits) * 4,  # R and W (float32)
@@ -254,7 +255,7 @@ class Layers:
     instances (their own K, V, codes, metadata, R, W, query and outputs), so
     that a cycle over them touches more than L2, and one workspace."""
 
-    def __init__(self, w, inp, n, dev):
+    def __init__(self, w, inp, n, dev, flags=0):
         import numpy as np
         import torch
         import kv_cache_retrieval_b200 as hhr
@@ -263,12 +264,13 @@ class Layers:
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
 
         self.w, self.dev = w, dev
-        self.dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap)
+        self.dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap, flags)
         K0, V0 = bf(inp.K), bf(inp.V)
         R0, W0 = torch.from_numpy(inp.R).to(dev), torch.from_numpy(inp.W).to(dev)
         self.q_all = bf(inp.q)                       # [steps][B][Hq][d]
         codes0 = torch.zeros(w.B, w.Hkv, w.n_cap, w.words, dtype=torch.int32, device=dev)
-        meta0 = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=torch.bfloat16, device=dev)
+        meta_dtype = torch.float32 if flags & hhr.HHR_FLAG_META_F32 else torch.bfloat16
+        meta0 = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=meta_dtype, device=dev)
         hhr.hhr_encode_keys(self.dims, K0, R0, W0, 0, w.N, codes0, meta0)
         self.lay = []
         for li in range(n):
@@ -353,18 +355,20 @@ def encode_ms(lay, w, reps=5):
     return e0.elapsed_time(e1) / reps
 
 
-def workload_line(name, steps, warmup, dev, peak):
+def workload_line(name, steps, warmup, dev, peak, flags=0):
     """One secondary workload: device µs per step (its appends inside the
     timed steps when it has any), the roofline fraction of its algorithmic
-    bytes, its key encoding and the planted-key recall."""
+    bytes, its key encoding and the planted-key recall.  flags: the
+    hhr_dims variant flags (float32 metadata, GQA-sum)."""
     import torch
     import kv_cache_retrieval_b200 as hhr
     from workloads import get, make_inputs
     w = get(name)
     inp = make_inputs(w)
-    per_step = algorithmic_bytes(w, w.N, w.P, w.k)[1]
+    meta_bytes = 4 if flags & hhr.HHR_FLAG_META_F32 else 2
+    per_step = algorithmic_bytes(w, w.N, w.P, w.k, meta_bytes)[1]
     n_layers = max(1, min(12, int(math.ceil(2.2 * 126e6 / max(per_step, 1)))))   # > 2x L2 per cycle
-    lay = Layers(w, inp, n_layers, dev)
+    lay = Layers(w, inp, n_layers, dev, flags)
     enc = encode_ms(lay, w)
     if w.appends:
         # one step = append the next key, then decode with it (the graph
@@ -374,7 +378,7 @@ def workload_line(name, steps, warmup, dev, peak):
                 lay.append(0, i, stream)
                 lay.step(0, stream, n_valid=w.N + i + 1, q=lay.q_all[i])
         us, n, launch = graph_time_us(body, w.appends, steps, warmup)
-        per_step = algorithmic_bytes(w, w.N + w.appends, w.P, w.k)[1]
+        per_step = algorithmic_bytes(w, w.N + w.appends, w.P, w.k, meta_bytes)[1]
     else:
         def body(stream):
             for li in range(n_layers):
@@ -389,11 +393,56 @@ def workload_line(name, steps, warmup, dev, peak):
         recall = {"error": f"{type(exc).__name__}: {exc}"}
     achieved = per_step / (us * 1e-6) / 1e9
     out = {"us_per_step": round(us, 3), "steps": n, "layers_cycled": n_layers, "launch": launch,
+           "P": w.P, "k": w.k, "flags": flags,
            "appends_in_step": bool(w.appends), "algorithmic_bytes": per_step,
            "achieved_gbs": round(achieved, 1), "frac": round(achieved / peak, 4),
            "frac_vs_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
            "keys_scored_per_s": w.B * w.Hkv * w.N / (us * 1e-6),
            "encode_ms": round(enc, 4), "planted_recall": recall, "status": hhr.hhr_status_string(st)}
+    del lay, inp
+    torch.cuda.empty_cache()
+    return out
+
+
+def dense_sweep_line(N, steps, warmup, dev, peak):
+    """Decode speed of HHR over dense attention at context N (the comparison
+    of §4.3 "Context Length", Fig. 7, on synthetic Llama-shaped inputs): the
+    fused HHR step with the paper's ratios (candidate budget 30% of the
+    pages, Top-K 1.5% of the keys; Appendix A, §4.1) against
+    hhr_dense_attend over every key, both device-timed in CUDA graphs over
+    layer instances that together exceed L2."""
+    import torch
+    import kv_cache_retrieval_b200 as hhr
+    from workloads import get, make_inputs, scaled
+    base = get("llama8b_128k")
+    NP = (N + base.page - 1) // base.page
+    w = scaled(base, name=f"llama8b_{N // 1024}k_paper", N=N, P=max(1, round(0.3 * NP)),
+               k=max(1, round(0.015 * N)))
+    inp = make_inputs(w)
+    units = w.B * w.Hkv
+    dense_bytes = units * N * 2 * w.d * 2 + w.B * w.Hq * w.d * (2 + 4)
+    hhr_bytes = algorithmic_bytes(w, N, w.P, w.k)[1]
+    n_layers = max(1, min(12, int(math.ceil(2.2 * 126e6 / hhr_bytes))))
+    lay = Layers(w, inp, n_layers, dev)
+
+    def body_hhr(stream):
+        for li in range(n_layers):
+            lay.step(li, stream)
+
+    def body_dense(stream):
+        for li in range(n_layers):
+            L = lay.lay[li]
+            hhr.hhr_dense_attend(lay.dims, L["q"], L["K"], L["V"], w.N, lay.scale, L["out"], lay.ws, None,
+                                 stream)
+
+    us_h, n_h, _ = graph_time_us(body_hhr, n_layers, steps, warmup)
+    us_d, n_d, _ = graph_time_us(body_dense, n_layers, max(n_layers, steps // 4), warmup)
+    st = hhr.hhr_read_status(lay.ws)
+    out = {"N": N, "P": w.P, "k": w.k, "layers_cycled": n_layers, "hhr_us": round(us_h, 3),
+           "dense_us": round(us_d, 3), "speedup": round(us_d / us_h, 3),
+           "hhr_frac": round(hhr_bytes / (us_h * 1e-6) / 1e9 / peak, 4),
+           "dense_frac": round(dense_bytes / (us_d * 1e-6) / 1e9 / peak, 4),
+           "status": hhr.hhr_status_string(st)}
     del lay, inp
     torch.cuda.empty_cache()
     return out
@@ -540,14 +589,32 @@ def run_hhr(args):
         del lay, graphs
         torch.cuda.empty_cache()
         workloads = {}
-        for name in ("tiny_4k", "llama8b_32k", "batch8_64k_b256", "qwen8b_128k_rope"):
-            if name == w.name:
+        # the other workloads, the paper's budget ratios at 128K, and the two
+        # reading variants at 128K (float32 metadata, GQA-sum distances)
+        lines = [(n, n, 0) for n in ("tiny_4k", "llama8b_32k", "batch8_64k_b256", "qwen8b_128k_rope",
+                                     "llama8b_128k_paper")]
+        lines += [("llama8b_128k meta_f32", "llama8b_128k", hhr.HHR_FLAG_META_F32),
+                  ("llama8b_128k gqa_sum", "llama8b_128k", hhr.HHR_FLAG_GQA_SUM)]
+        for label, name, flags in lines:
+            if name == w.name and not flags:
                 continue
             try:
-                workloads[name] = workload_line(name, args.workload_steps, 20, dev, peak)
+                workloads[label] = workload_line(name, args.workload_steps, 20, dev, peak, flags)
             except Exception as exc:  # noqa: BLE001 - a secondary line must not cost the headline
-                workloads[name] = {"error": f"{type(exc).__name__}: {exc}"}
+                workloads[label] = {"error": f"{type(exc).__name__}: {exc}"}
             torch.cuda.empty_cache()
+        sweep = {}
+        for N in (16384, 32768, 65536, 131072):
+            try:
+                sweep[f"{N // 1024}k"] = dense_sweep_line(N, args.workload_steps, 20, dev, peak)
+            except Exception as exc:  # noqa: BLE001
+                sweep[f"{N // 1024}k"] = {"error": f"{type(exc).__name__}: {exc}"}
+            torch.cuda.empty_cache()
+        workloads["dense_comparison"] = {
+            "what": "decode step of HHR (paper ratios: 30% pages, 1.5% keys) vs dense decode "
+                    "attention over every key; speedup = dense_us / hhr_us (the paper's Fig. 7 "
+                    "reports 1.16x at 16K to 3.30x at 128K on A800, context only)",
+            "by_context": sweep}
 
     if rank == 0:
         line = {

@@ -203,6 +203,21 @@ int32_t hhr_sparse_attend(const hhr_dims* dims, const void* q, const void* K, co
                           void* stream);
 
 /*
+ * Dense decode attention, the comparator the paper measures HHR against
+ * (§4.3 "Context Length", Fig. 7: decode speed of HHR over full attention):
+ * out[b][h] = sum_n softmax_n(scale * q[b][h].K[b][g][n]) V[b][g][n] over
+ * every key n < n_valid of the head's KV group g, float32 accumulation of the
+ * bf16 inputs.  n_valid == 0 gives zeros.  Same kernels and merge as
+ * hhr_sparse_attend, over contiguous key ranges (each CTA one range).
+ *   q, K, V  device, read; out device, write (layouts above).
+ *   n_valid  0 <= n_valid <= n_cap.
+ *   workspace as for hhr_sparse_attend (hhr_workspace_size(dims, 1, 1)).
+ */
+int32_t hhr_dense_attend(const hhr_dims* dims, const void* q, const void* K, const void* V,
+                         int32_t n_valid, float scale, float* out, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/*
  * One fused decode step: hhr_select followed by hhr_sparse_attend, in a
  * single launch.  Arguments as for those two calls.
  */

@@ -11,7 +11,7 @@ CUDA kernels.  This package is its ctypes binding (same function names) plus
 """
 from ._binding import (HHR_ERR_CUDA, HHR_ERR_INVALID_ARG, HHR_ERR_TIMEOUT, HHR_ERR_UNSUPPORTED,
                        HHR_ERR_WORKSPACE, HHR_FLAG_GQA_SUM, HHR_FLAG_META_F32, HHR_MAX_PAGES,
-                       HHR_OK, HhrError, hhr_decode_step, hhr_decode_step_host,
+                       HHR_OK, HhrError, hhr_decode_step, hhr_decode_step_host, hhr_dense_attend,
                        hhr_decode_step_noalloc, hhr_dims, hhr_encode_keys, hhr_encode_status,
                        hhr_noalloc_read_status, hhr_read_status, hhr_select, hhr_sparse_attend,
                        hhr_status_string, hhr_test_arm_timeout, hhr_version, hhr_workspace_size,
@@ -22,5 +22,5 @@ __all__ = [
     "HHR_OK", "HHR_ERR_INVALID_ARG", "HHR_ERR_UNSUPPORTED", "HHR_ERR_WORKSPACE", "HHR_ERR_CUDA",
     "HHR_ERR_TIMEOUT", "HHR_MAX_PAGES", "HHR_FLAG_META_F32", "HHR_FLAG_GQA_SUM", "HhrError", "hhr_dims", "make_dims", "lib", "hhr_version",
     "hhr_status_string", "hhr_encode_keys", "hhr_encode_status", "hhr_workspace_size", "hhr_select",
-    "hhr_sparse_attend", "hhr_decode_step", "hhr_decode_step_host", "hhr_decode_step_noalloc", "hhr_noalloc_read_status", "hhr_read_status", "hhr_test_arm_timeout", "HHRCache",
+    "hhr_sparse_attend", "hhr_dense_attend", "hhr_decode_step", "hhr_decode_step_host", "hhr_decode_step_noalloc", "hhr_noalloc_read_status", "hhr_read_status", "hhr_test_arm_timeout", "HHRCache",
 ]

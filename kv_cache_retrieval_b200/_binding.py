@@ -60,6 +60,8 @@ _SIGS = {
                           _P, _P, _P, C.c_size_t, _P]),
     "hhr_sparse_attend": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _I32, C.c_float, _P, _P,
                                  C.c_size_t, _P]),
+    "hhr_dense_attend": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _I32, C.c_float, _P, _P, C.c_size_t,
+                                _P]),
     "hhr_decode_step": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32,
                                C.c_float, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "hhr_decode_step_host": (_I32, [C.POINTER(hhr_dims), _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
@@ -155,6 +157,13 @@ def hhr_sparse_attend(dims, q, K, V, tok_idx, n_sel, k, scale, out, workspace=No
     _check(lib().hhr_sparse_attend(C.byref(dims), _ptr(q), _ptr(K), _ptr(V), _ptr(tok_idx),
                                    _ptr(n_sel), k, scale, _ptr(out), _ptr(workspace), ws_bytes,
                                    _stream(stream)), "hhr_sparse_attend")
+
+
+def hhr_dense_attend(dims, q, K, V, n_valid, scale, out, workspace=None, ws_bytes=None,
+                     stream=None) -> None:
+    ws_bytes = _nbytes(workspace) if ws_bytes is None and workspace is not None else (ws_bytes or 0)
+    _check(lib().hhr_dense_attend(C.byref(dims), _ptr(q), _ptr(K), _ptr(V), n_valid, scale, _ptr(out),
+                                  _ptr(workspace), ws_bytes, _stream(stream)), "hhr_dense_attend")
 
 
 def hhr_decode_step(dims, q, R, W, codes, meta, K, V, n_valid, P, k, scale, page_idx, tok_idx,

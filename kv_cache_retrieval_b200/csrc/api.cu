@@ -80,7 +80,7 @@ int32_t device_info(DeviceInfo* info) {
 // Picks the CTAs per unit and fills the size fields of `a`.  Returns the
 // dynamic shared-memory bytes through *smem.
 int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, DecodeArgs* a,
-                    size_t* smem) {
+                    size_t* smem, bool dense = false) {
   DeviceInfo info;
   if (int32_t st = device_info(&info)) return st;
   const int r = d->Hq / d->Hkv;
@@ -93,7 +93,10 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   int C = resident / units;
   if (C < 1) C = 1;
   if (C > kMaxCtasPerUnit) C = kMaxCtasPerUnit;
-  if (mode == kModeAttend) {
+  if (dense) {
+    const int by_tokens = (n_valid + 255) / 256;  // at least 256 keys per CTA
+    if (C > by_tokens) C = by_tokens < 1 ? 1 : by_tokens;
+  } else if (mode == kModeAttend) {
     const int by_tokens = (k + 63) / 64;  // at least 64 tokens per CTA
     if (C > by_tokens) C = by_tokens < 1 ? 1 : by_tokens;
   } else {
@@ -107,7 +110,10 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   }
   int slice_pages = 0, slice_tokens = 0;
   for (;;) {
-    if (mode == kModeAttend) {
+    if (dense) {
+      slice_pages = 0;
+      slice_tokens = 1;   // no token list
+    } else if (mode == kModeAttend) {
       slice_pages = 0;
       slice_tokens = (k + C - 1) / C + 1;
     } else {
@@ -144,6 +150,7 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   a->meta_f32 = (d->flags & HHR_FLAG_META_F32) ? 1 : 0;
   a->gqa_sum = (d->flags & HHR_FLAG_GQA_SUM) ? 1 : 0;
   a->hbins = hbins;
+  a->dense = dense ? 1 : 0;
   *smem = lay.total;
   return HHR_OK;
 }
@@ -256,7 +263,7 @@ static int32_t decode_common(const hhr_dims* dims, int mode, const void* q, cons
                              int32_t n_valid, int32_t P, int32_t k, float scale, int32_t* page_idx,
                              int32_t* tok_idx, int32_t* n_sel, float* out, float* dbg_U,
                              int32_t* dbg_D, void* workspace, size_t ws_bytes, void* stream,
-                             bool check_only = false) {
+                             bool check_only = false, bool dense = false) {
   if (int32_t st = check_dims(dims)) return st;
   if (np_cap_of(dims) > HHR_MAX_PAGES) return HHR_ERR_UNSUPPORTED;
   if (k < 1 || !q) return HHR_ERR_INVALID_ARG;
@@ -270,13 +277,14 @@ static int32_t decode_common(const hhr_dims* dims, int mode, const void* q, cons
     if (!aligned16(K) || !aligned16(V)) return HHR_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return HHR_ERR_INVALID_ARG;
   }
-  if (mode == kModeAttend && (!tok_in || !nsel_in)) return HHR_ERR_INVALID_ARG;
+  if (mode == kModeAttend && !dense && (!tok_in || !nsel_in)) return HHR_ERR_INVALID_ARG;
+  if (dense && (n_valid < 0 || n_valid > dims->n_cap)) return HHR_ERR_INVALID_ARG;
   if (int32_t st = check_workspace(dims, workspace, ws_bytes)) return st;
 
   DecodeArgs a;
   std::memset(&a, 0, sizeof a);
   size_t smem = 0;
-  if (int32_t st = plan_decode(dims, mode, n_valid, P, k, &a, &smem)) return st;
+  if (int32_t st = plan_decode(dims, mode, n_valid, P, k, &a, &smem, dense)) return st;
   if (check_only) return HHR_OK;
   a.q = static_cast<const uint16_t*>(q);
   a.R = R;
@@ -321,6 +329,14 @@ int32_t hhr_sparse_attend(const hhr_dims* dims, const void* q, const void* K, co
   return decode_common(dims, kModeAttend, q, nullptr, nullptr, nullptr, nullptr, K, V, tok_idx,
                        n_sel, dims ? dims->n_cap : 0, 1, k, scale, nullptr, nullptr, nullptr, out,
                        nullptr, nullptr, workspace, ws_bytes, stream);
+}
+
+int32_t hhr_dense_attend(const hhr_dims* dims, const void* q, const void* K, const void* V,
+                         int32_t n_valid, float scale, float* out, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  return decode_common(dims, kModeAttend, q, nullptr, nullptr, nullptr, nullptr, K, V, nullptr,
+                       nullptr, n_valid, 1, 1, scale, nullptr, nullptr, nullptr, out, nullptr, nullptr,
+                       workspace, ws_bytes, stream, false, true);
 }
 
 int32_t hhr_decode_step(const hhr_dims* dims, const void* q, const float* R, const float* W,

@@ -42,6 +42,7 @@
 
 #include <cfloat>
 #include <cstdint>
+#include <type_traits>
 
 #include "hhr_internal.cuh"
 
@@ -458,10 +459,11 @@ __device__ __forceinline__ void merge_states(const float* o, const float* ml, in
 //               rows 8-15 = the bf16 remainder, so P loses no precision.
 // Online softmax in float32 (exp2 with the scale folded in).  The next
 // tile's K is fetched during the softmax and P V, its V during the next Q K^T.
-template <int RG>
+template <int RG, bool kDense = false>
 __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const int* sel, int cnt,
                                   const float* qf,
-                                  unsigned char* scratch, uint32_t final_target, int* s_int) {
+                                  unsigned char* scratch, uint32_t final_target, int* s_int,
+                                  int dense0 = 0) {
   static_assert(RG <= 8, "the heads fill at most the upper 8 rows of an m16 tile");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, t4 = lane & 3;      // mma fragment: row (head), column pair
@@ -485,7 +487,9 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
         const int r = (lane >> 4) + 2 * i;
         const int t = tile * 16 + r;
         const bool ok = t < cnt;
-        const uint16_t* src = ok ? base + static_cast<size_t>(sel[t]) * kD + ch * 8 : base;
+        // the token: sel[t], or dense0 + t without a list (dense attention)
+        const int tok = kDense ? dense0 + t : (ok ? sel[t] : 0);
+        const uint16_t* src = ok ? base + static_cast<size_t>(tok) * kD + ch * 8 : base;
         cp_async16_zfill(buf + r * 256 + ((ch ^ (r & 7)) << 4), src, ok ? 16u : 0u);
       }
     }
@@ -735,6 +739,16 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
     const uint16_t* qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * RG) * kD;
 
     if constexpr (MODE == kModeAttend) {
+      if (a.dense) {
+        // dense attention over all n_valid keys: this CTA's contiguous
+        // share, c * n / C .. (c + 1) * n / C (c * n < 2^26: n <= HHR_MAX_PAGES * 64)
+        const int n = a.n_valid;
+        const int s0 = c * n / a.C, s1 = (c + 1) * n / a.C;
+        attend_and_finish<RG, true>(a, unit, c, nullptr, s1 - s0, nullptr, S.scratch, static_cast<uint32_t>(a.C),
+                              s_misc, s0);
+        __syncthreads();
+        continue;
+      }
       const int n = a.nsel_in[unit];
       const int s0 = c * n / a.C;         // c * n < 2^26 (n <= C * kMaxTokensPerCta)
       const int s1 = (c + 1) * n / a.C;
@@ -1308,42 +1322,49 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       __syncthreads();
       const uint32_t* codes_u = a.codes + static_cast<size_t>(unit) * a.n_cap * WORDS;
       int32_t* dbgD = a.dbg_D ? a.dbg_D + static_cast<size_t>(unit) * a.P * S_ : nullptr;
-      for (int i0 = warp * 32; i0 < ntok; i0 += NT) {
-        const int i = i0 + lane;
-        int D = 0xFFFF;
-        int slot = 0, off = 0;
-        if (i < ntok) {
-          slot = i / S_;
-          off = i - slot * S_;
-          const long long n = static_cast<long long>(S.my_pages[slot]) * S_ + off;
-          if (n < a.n_valid) {
-            uint32_t kc[WORDS];
-            const uint4* cp = reinterpret_cast<const uint4*>(codes_u + n * WORDS);
-#pragma unroll
-            for (int w4 = 0; w4 < WORDS / 4; ++w4) {
-              const uint4 t = __ldcs(cp + w4);
-              kc[w4 * 4 + 0] = t.x;
-              kc[w4 * 4 + 1] = t.y;
-              kc[w4 * 4 + 2] = t.z;
-              kc[w4 * 4 + 3] = t.w;
+      // the token loop, specialised on the group aggregation
+      auto hamming_pass = [&](auto sum_tag) {
+        constexpr bool kSum = decltype(sum_tag)::value;
+        for (int i0 = warp * 32; i0 < ntok; i0 += NT) {
+          const int i = i0 + lane;
+          int D = 0xFFFF;
+          int slot = 0, off = 0;
+          if (i < ntok) {
+            slot = i / S_;
+            off = i - slot * S_;
+            const long long n = static_cast<long long>(S.my_pages[slot]) * S_ + off;
+            if (n < a.n_valid) {
+              uint32_t kc[WORDS];
+              const uint4* cp = reinterpret_cast<const uint4*>(codes_u + n * WORDS);
+  #pragma unroll
+              for (int w4 = 0; w4 < WORDS / 4; ++w4) {
+                const uint4 t = __ldcs(cp + w4);
+                kc[w4 * 4 + 0] = t.x;
+                kc[w4 * 4 + 1] = t.y;
+                kc[w4 * 4 + 2] = t.z;
+                kc[w4 * 4 + 3] = t.w;
+              }
+              int agg = kSum ? 0 : 1 << 20;   // Eq. 2 over the group: min, or sum (GQA-sum)
+  #pragma unroll
+              for (int h = 0; h < RG; ++h) {
+                int dist = 0;
+  #pragma unroll
+                for (int w = 0; w < WORDS; ++w) dist += __popc(qc[h][w] ^ kc[w]);
+                agg = kSum ? agg + dist : min(agg, dist);
+              }
+              D = agg;
             }
-            int best = 1 << 20, total = 0;
-#pragma unroll
-            for (int h = 0; h < RG; ++h) {
-              int dist = 0;
-#pragma unroll
-              for (int w = 0; w < WORDS; ++w) dist += __popc(qc[h][w] ^ kc[w]);
-              best = min(best, dist);
-              total += dist;
-            }
-            D = a.gqa_sum ? total : best;   // Eq. 2 over the group: min, or sum (GQA-sum)
+            S.tokD[i] = static_cast<uint16_t>(D);
+            if (dbgD) dbgD[static_cast<size_t>(ks + slot) * S_ + off] = (D == 0xFFFF) ? -1 : D;
           }
-          S.tokD[i] = static_cast<uint16_t>(D);
-          if (dbgD) dbgD[static_cast<size_t>(ks + slot) * S_ + off] = (D == 0xFFFF) ? -1 : D;
+          const unsigned grp = __match_any_sync(0xFFFFFFFFu, D);
+          if (D != 0xFFFF && lane == __ffs(grp) - 1) atomicAdd(&sHD[D], __popc(grp));
         }
-        const unsigned grp = __match_any_sync(0xFFFFFFFFu, D);
-        if (D != 0xFFFF && lane == __ffs(grp) - 1) atomicAdd(&sHD[D], __popc(grp));
-      }
+      };
+      if (a.gqa_sum)
+        hamming_pass(std::true_type{});
+      else
+        hamming_pass(std::false_type{});
       if (c == 0 && dbgD)
         for (int i = Pk * S_ + tid; i < a.P * S_; i += NT) dbgD[i] = -1;
       __syncthreads();
@@ -1378,101 +1399,130 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // warp 0 alone finds the threshold distance T (the k_eff-th smallest),
       // how many tokens at T are still needed, and each CTA's tie quota and
       // output offset in CTA order.
-      const int VPL = (HB + 1 + 31) / 32;
-      int* sPre = sHA + a.C * HB;                        // [C][HB + 1]
-      int* sTot = sPre + a.C * (HB + 1);                 // [HB]
-      for (int cc = warp; cc < a.C; cc += NWARPS) {
-        const int* row = sHA + cc * HB;
-        const int v0 = lane * VPL, v1 = min(v0 + VPL, HB);
-        int loc = 0;
-        for (int v = v0; v < v1; ++v) loc += row[v];
-        int incl = loc;
+      // VPLC: bins per lane known at compile time (the min distances, HB =
+      // BITS + 1: loops unrolled, loads batched); 0: sized at run time
+      // (GQA-sum, HB up to r BITS + 1)
+      auto threshold = [&](auto vpl_tag) {
+        constexpr int VPLC = decltype(vpl_tag)::value;
+        const int HB = VPLC ? BITS + 1 : a.hbins;       // a compile-time constant with VPLC
+        const int VPL = VPLC ? VPLC : (HB + 1 + 31) / 32;
+        int* sPre = sHA + a.C * HB;                      // [C][HB + 1]
+        int* sTot = sPre + a.C * (HB + 1);               // [HB]
+        for (int cc = warp; cc < a.C; cc += NWARPS) {
+          const int* row = sHA + cc * HB;
+          const int v0 = lane * VPL;
+          // compile-time bins: the lane's counts in registers, all loaded
+          // before the first store (a store to sPre would otherwise order
+          // every later load of row behind it)
+          int hv[VPLC ? VPLC : 1];
+          int loc = 0;
 #pragma unroll
-        for (int o2 = 1; o2 < 32; o2 <<= 1) {
-          const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
-          if (lane >= o2) incl += y;
-        }
-        int run = incl - loc;
-        for (int v = v0; v < v1; ++v) {
-          sPre[cc * (HB + 1) + v] = run;
-          run += row[v];
-        }
-        if (v0 <= HB && HB < v0 + VPL) sPre[cc * (HB + 1) + HB] = run;   // the row's total
-      }
-      for (int v = tid; v < HB; v += NT) {
-        int x = 0;
-#pragma unroll 6
-        for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * HB + v];
-        sTot[v] = x;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        const int v0 = lane * VPL, v1 = min(v0 + VPL, HB);
-        int loc = 0;
-        for (int v = v0; v < v1; ++v) loc += sTot[v];
-        int incl = loc;
+          for (int e = 0; e < (VPLC ? VPLC : VPL); ++e) {
+            const int x = v0 + e < HB ? row[v0 + e] : 0;
+            if (VPLC) hv[VPLC ? e : 0] = x;
+            loc += x;
+          }
+          int incl = loc;
 #pragma unroll
-        for (int o2 = 1; o2 < 32; o2 <<= 1) {
-          const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
-          if (lane >= o2) incl += y;
-        }
-        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        const int k_eff = min(a.k, total);
-        // the lane whose bins hold the k_eff-th smallest distance
-        int T = -1, needT = 0;
-        if (incl - loc < k_eff && incl >= k_eff) {
+          for (int o2 = 1; o2 < 32; o2 <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
+            if (lane >= o2) incl += y;
+          }
           int run = incl - loc;
-          for (int v = v0; v < v1; ++v) {
-            const int xv = sTot[v];
-            if (run < k_eff && run + xv >= k_eff) {
-              T = v;
-              needT = k_eff - run;
+#pragma unroll
+          for (int e = 0; e < (VPLC ? VPLC : VPL); ++e) {
+            const int v = v0 + e;
+            if (v < HB) {
+              sPre[cc * (HB + 1) + v] = run;
+              run += VPLC ? hv[VPLC ? e : 0] : row[v];
+            } else if (v == HB) {
+              sPre[cc * (HB + 1) + HB] = run;   // the row's total
             }
-            run += xv;
           }
         }
-        const unsigned own = __ballot_sync(0xFFFFFFFFu, T >= 0);
-        if (own) {
-          const int src = __ffs(own) - 1;
-          T = __shfl_sync(0xFFFFFFFFu, T, src);
-          needT = __shfl_sync(0xFFFFFFFFu, needT, src);
+        for (int v = tid; v < HB; v += NT) {
+          int x = 0;
+#pragma unroll 6
+          for (int cc = 0; cc < a.C; ++cc) x += sHA[cc * HB + v];
+          sTot[v] = x;
         }
-        int pre_eq = 0, off = 0;
-        for (int c0 = 0; c0 < a.C; c0 += 32) {   // CTAs in order: tie quota and output offset
-          const int cc = c0 + lane;
-          int below = 0, eq = 0;
-          if (cc < a.C && T >= 0) {
-            below = sPre[cc * (HB + 1) + T];
-            eq = sPre[cc * (HB + 1) + T + 1] - below;
-          }
-          int eq_in = eq;
+        __syncthreads();
+        if (warp == 0) {
+          const int v0 = lane * VPL;
+          int loc = 0;
+#pragma unroll
+          for (int e = 0; e < (VPLC ? VPLC : VPL); ++e)
+            if (v0 + e < HB) loc += sTot[v0 + e];
+          int incl = loc;
 #pragma unroll
           for (int o2 = 1; o2 < 32; o2 <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, eq_in, o2);
-            if (lane >= o2) eq_in += y;
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
+            if (lane >= o2) incl += y;
           }
-          const int quota = max(0, min(needT - (pre_eq + eq_in - eq), eq));
-          const int selc = below + quota;
-          int sel_in = selc;
+          const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+          const int k_eff = min(a.k, total);
+          // the lane whose bins hold the k_eff-th smallest distance
+          int T = -1, needT = 0;
+          if (incl - loc < k_eff && incl >= k_eff) {
+            int run = incl - loc;
 #pragma unroll
-          for (int o2 = 1; o2 < 32; o2 <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, sel_in, o2);
-            if (lane >= o2) sel_in += y;
+            for (int e = 0; e < (VPLC ? VPLC : VPL); ++e) {
+              const int v = v0 + e;
+              const int xv = v < HB ? sTot[v] : 0;
+              if (run < k_eff && run + xv >= k_eff) {
+                T = v;
+                needT = k_eff - run;
+              }
+              run += xv;
+            }
           }
-          if (cc == c) {
-            s_misc[7] = off + sel_in - selc;
-            s_misc[8] = quota;
-            s_misc[9] = selc;
+          const unsigned own = __ballot_sync(0xFFFFFFFFu, T >= 0);
+          if (own) {
+            const int src = __ffs(own) - 1;
+            T = __shfl_sync(0xFFFFFFFFu, T, src);
+            needT = __shfl_sync(0xFFFFFFFFu, needT, src);
           }
-          pre_eq += __shfl_sync(0xFFFFFFFFu, eq_in, 31);
-          off += __shfl_sync(0xFFFFFFFFu, sel_in, 31);
+          int pre_eq = 0, off = 0;
+          for (int c0 = 0; c0 < a.C; c0 += 32) {   // CTAs in order: tie quota and output offset
+            const int cc = c0 + lane;
+            int below = 0, eq = 0;
+            if (cc < a.C && T >= 0) {
+              below = sPre[cc * (HB + 1) + T];
+              eq = sPre[cc * (HB + 1) + T + 1] - below;
+            }
+            int eq_in = eq;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+              const int y = __shfl_up_sync(0xFFFFFFFFu, eq_in, o2);
+              if (lane >= o2) eq_in += y;
+            }
+            const int quota = max(0, min(needT - (pre_eq + eq_in - eq), eq));
+            const int selc = below + quota;
+            int sel_in = selc;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+              const int y = __shfl_up_sync(0xFFFFFFFFu, sel_in, o2);
+              if (lane >= o2) sel_in += y;
+            }
+            if (cc == c) {
+              s_misc[7] = off + sel_in - selc;
+              s_misc[8] = quota;
+              s_misc[9] = selc;
+            }
+            pre_eq += __shfl_sync(0xFFFFFFFFu, eq_in, 31);
+            off += __shfl_sync(0xFFFFFFFFu, sel_in, 31);
+          }
+          if (lane == 0) {
+            s_misc[5] = T;
+            s_misc[6] = k_eff;
+          }
         }
-        if (lane == 0) {
-          s_misc[5] = T;
-          s_misc[6] = k_eff;
-        }
-      }
-      __syncthreads();
+        __syncthreads();
+      };
+      if (a.gqa_sum)
+        threshold(std::integral_constant<int, 0>{});
+      else
+        threshold(std::integral_constant<int, (BITS + 2 + 31) / 32>{});
       const int T = s_misc[5], k_eff = s_misc[6];
       const int my_off = s_misc[7], my_quota = s_misc[8], my_sel = s_misc[9];
       {

@@ -93,6 +93,7 @@ struct DecodeArgs {
   int meta_f32;             // HHR_FLAG_META_F32: f32 metadata, bounds by SIMT
   int gqa_sum;              // HHR_FLAG_GQA_SUM: distance = sum over the group's heads
   int hbins;                // distance histogram bins (hist_bins)
+  int dense;                // attend mode over all n_valid keys, no token list (hhr_dense_attend)
 };
 
 struct EncodeArgs {

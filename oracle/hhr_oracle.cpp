@@ -340,6 +340,25 @@ int64_t hhro_top_tokens(const int32_t* D, const int32_t* pages, int64_t n_pages,
   return cnt;
 }
 
+// Selection-quality reference (diagnostic): the m keys among [0, n_valid)
+// with the largest exact group logit max_h q_h . k_n (double, from the bf16
+// values; the same "any head of the group" reading as R4), ties to the lower
+// index, written ascending.  Returns the count.  K: [n_cap][d] bf16 bits.
+int64_t hhro_top_logits(const uint16_t* q, int32_t r, int32_t d, const uint16_t* K, int64_t n_valid,
+                        int64_t m, int32_t* out) {
+  std::vector<double> s(static_cast<size_t>(n_valid));
+  for (int64_t n = 0; n < n_valid; ++n) {
+    double best = -std::numeric_limits<double>::infinity();
+    for (int h = 0; h < r; ++h) {
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j) acc += widen_bf16(q[h * d + j]) * widen_bf16(K[n * d + j]);
+      best = std::max(best, acc);
+    }
+    s[n] = best;
+  }
+  return hhro_top_largest(s.data(), n_valid, m, out);
+}
+
 // Attention over the selected keys (§1: attention is computed on the keys the
 // hash retrieval selects; reading R7).  For each of the r heads:
 // s_i = scale * q_h . K[idx_i], o = sum_i e^(s_i - max s) V[idx_i] / sum_i e^(s_i - max s).

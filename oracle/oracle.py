@@ -46,6 +46,7 @@ def lib():
             "hhro_decode_unit": (i64, [p, i32, i32, i32, i32, p, p, p, p, p, p,
                                        i64, i64, i64, f64, p, p, p, p, p, p]),
             "hhro_page_meta_f32": (None, [p, i64, i64, i32, i32, i64, i64, p]),
+            "hhro_top_logits": (i64, [p, i32, i32, p, i64, i64, p]),
             "hhro_encode_unit_f32": (i64, [p, i64, i64, i32, i32, i32, p, p, p, p]),
             "hhro_page_bounds_f32": (None, [p, i32, i32, p, i64, p, p]),
             "hhro_hamming_agg": (None, [p, i32, i32, p, p, i64, i32, i64, i32, p]),
@@ -168,6 +169,16 @@ def top_tokens(D, pages, page, k):
     pages = _c(pages, np.int32)
     out = np.empty(k, np.int32)
     cnt = lib().hhro_top_tokens(_p(D), _p(pages), pages.shape[0], page, k, _p(out))
+    return out[:cnt]
+
+
+def top_logits(q_bits, K_unit, n_valid, m):
+    """Diagnostic reference: the m keys of [0, n_valid) with the largest exact
+    group logit max_h q_h . k_n, ties to the lower index, ascending."""
+    q = _c(q_bits, np.uint16)
+    r, d = q.shape
+    out = np.empty(min(m, n_valid), np.int32)
+    cnt = lib().hhro_top_logits(_p(q), r, d, _p(_c(K_unit, np.uint16)), n_valid, m, _p(out))
     return out[:cnt]
 
 

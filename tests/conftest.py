@@ -33,9 +33,13 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     parity rules allow (near-cutoff pages, ambiguous query bits), and how the
     attention outputs were checked."""
     try:
-        from gpu_harness import REPORTS
+        from gpu_harness import QUALITY, REPORTS
     except Exception:  # noqa: BLE001 - the harness needs torch + CUDA
         return
+    if QUALITY:
+        terminalreporter.write_sep("-", "selection quality (diagnostic): recall of the exact top-k by logit")
+        for q in QUALITY:
+            terminalreporter.write_line(str(q))
     if not REPORTS:
         return
     keys = ["units", "units_exact", "units_explained", "near_cutoff_pages", "tok_set_diff",

@@ -160,6 +160,10 @@ REPORTS = []
 
 MAX_PAGE_SWAPS = 2      # near-cutoff page swaps tolerated per unit
 
+# Selection-quality diagnostics (tests/test_selection_quality.py), printed in
+# the terminal summary.
+QUALITY = []
+
 
 def compare_select(w, ores, page_idx, tok_idx, n_sel, units, dbg_U=None, dbg_D=None, P=None,
                    k=None, inp=None, step=0, out_g=None, name=""):

@@ -136,3 +136,27 @@ def test_python_binding_raises_on_error_status():
     with pytest.raises(hhr.HhrError) as e:
         hhr.hhr_encode_keys(d, FAKE, FAKE, FAKE, 0, 1, FAKE, FAKE, stream=0)
     assert e.value.status == hhr.HHR_ERR_UNSUPPORTED
+
+
+def test_dense_attend_validation():
+    d = _dims()
+    L = hhr.lib()
+    ws = 1 << 30
+    assert L.hhr_dense_attend(C.byref(d), FAKE, FAKE, FAKE, 4097, C.c_float(0.1), FAKE, FAKE, ws,
+                              None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_dense_attend(C.byref(d), FAKE, FAKE, FAKE, -1, C.c_float(0.1), FAKE, FAKE, ws,
+                              None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_dense_attend(C.byref(d), FAKE, FAKE, FAKE, 10, C.c_float(float("inf")), FAKE, FAKE,
+                              ws, None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_dense_attend(C.byref(d), FAKE, FAKE, FAKE, 10, C.c_float(0.1), None, FAKE, ws,
+                              None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_dense_attend(C.byref(d), FAKE, FAKE, FAKE, 10, C.c_float(0.1), FAKE, None, ws,
+                              None) == hhr.HHR_ERR_WORKSPACE
+
+
+def test_variant_flags_validation():
+    assert _select(_dims(flags=4)) == hhr.HHR_ERR_INVALID_ARG
+    assert _select(_dims(flags=-1)) == hhr.HHR_ERR_INVALID_ARG
+    plain, summed = _dims(), _dims(flags=hhr.HHR_FLAG_GQA_SUM)
+    assert hhr.hhr_workspace_size(summed, 64, 256) > hhr.hhr_workspace_size(plain, 64, 256)
+    assert hhr.hhr_workspace_size(_dims(flags=8), 64, 256) == 0

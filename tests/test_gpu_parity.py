@@ -209,6 +209,33 @@ def test_variant_flags_are_validated():
     assert hhr.hhr_workspace_size(sumd, w.P, w.k) >= hhr.hhr_workspace_size(d.dims, w.P, w.k)
 
 
+# --------------------------------------------------------- dense comparator
+
+def _dense_ref(inp, units, n_valid, step=0):
+    w = inp.w
+    r = w.r
+    out = np.zeros((w.B, w.Hq, w.d), np.float32)
+    for (b, g) in units:
+        out[b, g * r:(g + 1) * r] = O.attend(inp.q[step, b, g * r:(g + 1) * r], inp.K[b, g], inp.V[b, g],
+                                             np.arange(n_valid, dtype=np.int32), 1.0 / np.sqrt(w.d))
+    return out
+
+
+@pytest.mark.parametrize("name,n_valid", [("tiny_4k", 4096), ("llama_20k_ragged", 20003),
+                                          ("gqa8", 3000), ("gqa2", 2999), ("b256_s32", 9001),
+                                          ("tiny_4k", 0), ("tiny_4k", 1), ("tiny_4k", 17)])
+def test_dense_attend_matches_oracle(name, n_valid):
+    """hhr_dense_attend = softmax attention over every valid key (the oracle's
+    attention with the full index list)."""
+    inp, _, _ = case(name)
+    w = inp.w
+    d = Dev(inp)
+    hhr.hhr_dense_attend(d.dims, d.q[0], d.K, d.V, n_valid, d.scale, d.out, d.ws)
+    assert d.status() == hhr.HHR_OK
+    err = compare_out(w, _dense_ref(inp, all_units(w), n_valid), _host(d.out), all_units(w))
+    print(name, n_valid, "dense max abs err", err)
+
+
 # ------------------------------------------------------------------ edge cases
 
 @pytest.mark.parametrize("n_valid", [0, 1, 5, 16, 17, 333, 4096])
@@ -417,3 +444,17 @@ def test_full_size_variants_sampled_units(variant):
     assert d.status() == hhr.HHR_OK
     torch.cuda.synchronize()
     compare_encode(inp, u32_host(d.codes), d.meta_host(), units, w.N)
+
+
+@pytest.mark.slow
+def test_full_size_dense_attend_sampled_units():
+    """The dense comparator at 128K in the launch configuration the benchmark
+    times (every unit runs; two are checked)."""
+    w = get("llama8b_128k")
+    inp = make_inputs(w)
+    units = [(0, 1), (0, 6)]
+    d = Dev(inp)
+    hhr.hhr_dense_attend(d.dims, d.q[0], d.K, d.V, w.N, d.scale, d.out, d.ws)
+    assert d.status() == hhr.HHR_OK
+    err = compare_out(w, _dense_ref(inp, units, w.N), _host(d.out), units)
+    print("dense 128K max abs err", err)

@@ -528,3 +528,19 @@ def test_decode_unit_variants_compose_the_primitives():
         assert res["tok_idx"][0, 0].tolist() == tok.tolist()
         assert res["D"][0, 0, :25 * 16].tolist() == D.tolist()
         assert np.array_equal(res["U"][(0, 0)], U)
+
+
+# ------------------------------------------- selection-quality reference
+
+def test_top_logits_matches_brute_force_ranking():
+    """The exact top-m keys by group logit (max over the heads of q_h . k):
+    numpy float64 logits and rank counting, ties to the lower index."""
+    rng = np.random.default_rng(26)
+    q = _rand_bits(rng, (4, 128))
+    k = _rand_bits(rng, (300, 128), 2.0)
+    k[50] = k[7]                     # an exact tie: the lower index wins
+    logits = (_f(q) @ _f(k).T).max(0)
+    for m in (1, 7, 40, 300, 500):
+        got = O.top_logits(q, k, 280, m)
+        assert got.tolist() == _rank_select(logits[:280], m, True)
+    assert 7 in O.top_logits(q[:, :], k, 280, 280).tolist()
