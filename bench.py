@@ -594,7 +594,9 @@ def run_hhr(args):
         lines = [(n, n, 0) for n in ("tiny_4k", "llama8b_32k", "batch8_64k_b256", "qwen8b_128k_rope",
                                      "llama8b_128k_paper")]
         lines += [("llama8b_128k meta_f32", "llama8b_128k", hhr.HHR_FLAG_META_F32),
-                  ("llama8b_128k gqa_sum", "llama8b_128k", hhr.HHR_FLAG_GQA_SUM)]
+                  ("llama8b_128k gqa_sum", "llama8b_128k", hhr.HHR_FLAG_GQA_SUM),
+                  # Eq. 3 on the CUDA cores instead of the tensor-core tiles (A/B)
+                  ("llama8b_128k simt_bounds", "llama8b_128k", hhr.HHR_FLAG_SIMT_BOUNDS)]
         for label, name, flags in lines:
             if name == w.name and not flags:
                 continue

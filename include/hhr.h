@@ -101,6 +101,9 @@ typedef enum hhr_status {
 /* hhr_dims.flags: variants of two readings (see the top of this file). */
 #define HHR_FLAG_META_F32 1  /* meta is f32, unrounded extrema               */
 #define HHR_FLAG_GQA_SUM 2   /* token distance = sum over the group's heads  */
+#define HHR_FLAG_SIMT_BOUNDS 4 /* Eq. 3 on the CUDA cores instead of the tensor
+                                  cores (bf16 metadata; same results up to
+                                  float32 rounding; for comparison)           */
 
 typedef struct hhr_dims {
   int32_t B;     /* sequences                                   */
@@ -110,7 +113,7 @@ typedef struct hhr_dims {
   int32_t bits;  /* code length b (128 or 256)                  */
   int32_t page;  /* tokens per page S                           */
   int32_t n_cap; /* KV-cache capacity per (sequence, KV head)   */
-  int32_t flags; /* 0, or HHR_FLAG_META_F32 | HHR_FLAG_GQA_SUM  */
+  int32_t flags; /* 0, or an OR of the HHR_FLAG_* above          */
 } hhr_dims;
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */

@@ -32,6 +32,7 @@ class HhrError(RuntimeError):
 
 HHR_FLAG_META_F32 = 1   # page metadata in float32 (unrounded extrema)
 HHR_FLAG_GQA_SUM = 2    # token distance = sum over the group's heads
+HHR_FLAG_SIMT_BOUNDS = 4  # Eq. 3 on the CUDA cores (comparison form of the tensor-core tiles)
 
 
 class hhr_dims(C.Structure):

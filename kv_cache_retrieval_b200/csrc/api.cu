@@ -28,7 +28,7 @@ int32_t check_dims(const hhr_dims* d) {
   if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->d < 1 || d->bits < 1 || d->page < 1 || d->n_cap < 1)
     return HHR_ERR_INVALID_ARG;
   if (d->Hq % d->Hkv != 0) return HHR_ERR_INVALID_ARG;
-  if (d->flags & ~(HHR_FLAG_META_F32 | HHR_FLAG_GQA_SUM)) return HHR_ERR_INVALID_ARG;
+  if (d->flags & ~(HHR_FLAG_META_F32 | HHR_FLAG_GQA_SUM | HHR_FLAG_SIMT_BOUNDS)) return HHR_ERR_INVALID_ARG;
   const int r = d->Hq / d->Hkv;
   if (d->d != kD) return HHR_ERR_UNSUPPORTED;
   if (d->bits != 128 && d->bits != 256) return HHR_ERR_UNSUPPORTED;
@@ -149,6 +149,7 @@ int32_t plan_decode(const hhr_dims* d, int mode, int n_valid, int P, int k, Deco
   a->spin_limit = kSpinLimit;
   a->meta_f32 = (d->flags & HHR_FLAG_META_F32) ? 1 : 0;
   a->gqa_sum = (d->flags & HHR_FLAG_GQA_SUM) ? 1 : 0;
+  a->simt_bounds = (d->flags & HHR_FLAG_SIMT_BOUNDS) ? 1 : 0;
   a->hbins = hbins;
   a->dense = dense ? 1 : 0;
   *smem = lay.total;

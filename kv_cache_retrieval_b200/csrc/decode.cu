@@ -935,6 +935,57 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           }
           issue_group(gi + GR);   // refill this lane's slots of group gi
         }
+      } else if (a.simt_bounds) {
+        // Eq. 3 on bf16 bounds on the CUDA cores (HHR_FLAG_SIMT_BOUNDS, the
+        // comparison form of the tensor-core tiles below): lane l holds the 8
+        // bf16 values of chunk l of a page -- dimensions 8 (l % 16) .. + 7 of
+        // the lower row (l < 16) or of the upper row -- and the matching
+        // min(q~, 0) or max(q~, 0) of every head; the warp sums the 32 lanes.
+        const int j0 = 8 * (lane & 15);
+        const bool upper = lane >= 16;
+        float qs[RG][8];
+#pragma unroll
+        for (int h = 0; h < RG; ++h)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float v = S.qt[h * kD + j0 + e];
+            qs[h][e] = upper ? fmaxf(v, 0.f) : fminf(v, 0.f);
+          }
+        for (int gi = 0; gi < n_grp; ++gi) {
+          cp_async_wait<GR - 1>();   // this lane's chunks of group gi have landed
+#pragma unroll 1
+          for (int pp = 0; pp < PPG; ++pp) {
+            const int pl = gi * PPG + pp;
+            if (pl >= w_pages) break;   // warp-uniform
+            const int sl = pl % kRingSlots;
+            const uint4 raw = ring[sl * (NWARPS * 32) + (lane ^ (sl & 7))];
+            const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              x[2 * e] = __uint_as_float(wv[e] << 16);
+              x[2 * e + 1] = __uint_as_float(wv[e] & 0xFFFF0000u);
+            }
+            float u = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < RG; ++h) {
+              float t = qs[h][0] * x[0];
+#pragma unroll
+              for (int e = 1; e < 8; ++e) t = fmaf(qs[h][e], x[e], t);
+#pragma unroll
+              for (int o2 = 16; o2 >= 1; o2 >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o2);
+              u = fmaxf(u, t);
+            }
+            if (lane == 0) {
+              const int pg = wpb + pl;
+              wsU_u[pg] = u;
+              if (a.dbg_U) a.dbg_U[static_cast<size_t>(unit) * a.NP + pg] = u;
+            }
+            lmin = fminf(lmin, u);
+            lmax = fmaxf(lmax, u);
+          }
+          issue_group(gi + GR);   // refill this lane's slots of group gi
+        }
       } else {
         for (int ti = 0; ti < n_tiles; ++ti) {
           cp_async_wait<1>();   // this lane's groups 2 ti and 2 ti + 1 have landed

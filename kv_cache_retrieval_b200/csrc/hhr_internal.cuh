@@ -94,6 +94,7 @@ struct DecodeArgs {
   int gqa_sum;              // HHR_FLAG_GQA_SUM: distance = sum over the group's heads
   int hbins;                // distance histogram bins (hist_bins)
   int dense;                // attend mode over all n_valid keys, no token list (hhr_dense_attend)
+  int simt_bounds;          // HHR_FLAG_SIMT_BOUNDS: Eq. 3 on the CUDA cores (bf16 metadata)
 };
 
 struct EncodeArgs {

@@ -155,8 +155,8 @@ def test_dense_attend_validation():
 
 
 def test_variant_flags_validation():
-    assert _select(_dims(flags=4)) == hhr.HHR_ERR_INVALID_ARG
+    assert _select(_dims(flags=8)) == hhr.HHR_ERR_INVALID_ARG
     assert _select(_dims(flags=-1)) == hhr.HHR_ERR_INVALID_ARG
     plain, summed = _dims(), _dims(flags=hhr.HHR_FLAG_GQA_SUM)
     assert hhr.hhr_workspace_size(summed, 64, 256) > hhr.hhr_workspace_size(plain, 64, 256)
-    assert hhr.hhr_workspace_size(_dims(flags=8), 64, 256) == 0
+    assert hhr.hhr_workspace_size(_dims(flags=16), 64, 256) == 0

@@ -151,6 +151,7 @@ VARIANTS = {
     "meta_f32": hhr.HHR_FLAG_META_F32,
     "gqa_sum": hhr.HHR_FLAG_GQA_SUM,
     "both": hhr.HHR_FLAG_META_F32 | hhr.HHR_FLAG_GQA_SUM,
+    "simt_bounds": hhr.HHR_FLAG_SIMT_BOUNDS,
 }
 _vcache = {}
 
@@ -200,7 +201,7 @@ def test_variant_flags_are_validated():
     inp, _, _ = case("tiny_4k")
     w = inp.w
     d = Dev(inp)
-    bad = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap, 4)
+    bad = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap, 8)
     with pytest.raises(hhr.HhrError) as e:
         hhr.hhr_encode_keys(bad, d.K, d.R, d.W, 0, w.N, d.codes, d.meta)
     assert e.value.status == hhr.HHR_ERR_INVALID_ARG
