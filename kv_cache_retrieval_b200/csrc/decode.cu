@@ -672,7 +672,9 @@ __device__ void attend_and_finish(const DecodeArgs& a, int unit, int c, const in
 }
 
 // ----------------------------------------------------------------------------
-template <int RG, int WORDS, int MODE>
+// VAR: the variant flags (float32 metadata, GQA-sum, SIMT bounds) may be set;
+// false compiles their branches out (every flag 0, the default readings).
+template <int RG, int WORDS, int MODE, bool VAR>
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_int[NWARPS + 16];
@@ -682,7 +684,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
   constexpr int BITS = WORDS * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x % a.C;
-  const DecodeSmem lay = decode_smem(a.NP, a.C, BITS, RG, a.slice_pages, a.slice_tokens, MODE, a.hbins);
+  // the variant flags, compile-time false without VAR
+  const bool meta_f32 = VAR && a.meta_f32, gqa_sum = VAR && a.gqa_sum, simt_bounds = VAR && a.simt_bounds;
+  const int hbins = VAR ? a.hbins : BITS + 1;
+  const DecodeSmem lay = decode_smem(a.NP, a.C, BITS, RG, a.slice_pages, a.slice_tokens, MODE, hbins);
   Smem S;
   S.qb = reinterpret_cast<uint16_t*>(smem + lay.qb);
   S.qf = reinterpret_cast<float*>(smem + lay.qf);
@@ -808,10 +813,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // bounds), PPG / 2 pages per group; lane l keeps chunk l of each half at
       // position l (it alone reads it back).
       const size_t meta_row = static_cast<size_t>(unit) * a.np_cap + wpb;   // first page of the warp
-      const uint4* wsrc = reinterpret_cast<const uint4*>(a.meta) + meta_row * (a.meta_f32 ? 64 : 32) + lane;
+      const uint4* wsrc = reinterpret_cast<const uint4*>(a.meta) + meta_row * (meta_f32 ? 64 : 32) + lane;
       uint4* ring = reinterpret_cast<uint4*>(S.scratch) + warp * 32;
       auto issue_group = [&](int gi) {  // every lane: its 16 B of each page half, one commit group
-        if (!a.meta_f32) {
+        if (!meta_f32) {
           if (gi < n_grp) {
 #pragma unroll
             for (int pp = 0; pp < PPG; ++pp) {
@@ -885,7 +890,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       const int g8 = lane >> 2, t4 = lane & 3;      // mma fragment: row, column pair
       const uint32_t ring_s = smem_addr(S.scratch) + warp * 512;
       const uint32_t qb_s = smem_addr(S.qb);
-      if (a.meta_f32) {
+      if (meta_f32) {
         // Eq. 3 on float32 bounds, on the CUDA cores: lane l holds dimensions
         // 4 l .. 4 l + 3 of a page's lower and upper bounds, forms
         // sum_j min(q~_hj, 0) l_j + max(q~_hj, 0) u_j over them for every head,
@@ -935,7 +940,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           }
           issue_group(gi + GR);   // refill this lane's slots of group gi
         }
-      } else if (a.simt_bounds) {
+      } else if (simt_bounds) {
         // Eq. 3 on bf16 bounds on the CUDA cores (HHR_FLAG_SIMT_BOUNDS, the
         // comparison form of the tensor-core tiles below): lane l holds the 8
         // bf16 values of chunk l of a page -- dimensions 8 (l % 16) .. + 7 of
@@ -1362,7 +1367,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // ---------------------------------------------------------- phase 4
       const int S_ = a.page;
       const int ntok = (ke - ks) * S_;
-      const int HB = a.hbins;                          // distance bins: BITS + 1, or r BITS + 1 (GQA-sum)
+      const int HB = hbins;                            // distance bins: BITS + 1, or r BITS + 1 (GQA-sum)
       int* sHD = reinterpret_cast<int*>(S.scratch);  // [HB]
       for (int i = tid; i < HB; i += NT) sHD[i] = 0;
       uint32_t qc[RG][WORDS];
@@ -1412,7 +1417,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
           if (D != 0xFFFF && lane == __ffs(grp) - 1) atomicAdd(&sHD[D], __popc(grp));
         }
       };
-      if (a.gqa_sum)
+      if (gqa_sum)
         hamming_pass(std::true_type{});
       else
         hamming_pass(std::false_type{});
@@ -1455,7 +1460,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // (GQA-sum, HB up to r BITS + 1)
       auto threshold = [&](auto vpl_tag) {
         constexpr int VPLC = decltype(vpl_tag)::value;
-        const int HB = VPLC ? BITS + 1 : a.hbins;       // a compile-time constant with VPLC
+        const int HB = VPLC ? BITS + 1 : hbins;         // a compile-time constant with VPLC
         const int VPL = VPLC ? VPLC : (HB + 1 + 31) / 32;
         int* sPre = sHA + a.C * HB;                      // [C][HB + 1]
         int* sTot = sPre + a.C * (HB + 1);               // [HB]
@@ -1570,7 +1575,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
         }
         __syncthreads();
       };
-      if (a.gqa_sum)
+      if (gqa_sum)
         threshold(std::integral_constant<int, 0>{});
       else
         threshold(std::integral_constant<int, (BITS + 2 + 31) / 32>{});
@@ -1628,9 +1633,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
   }
 }
 
-template <int RG, int WORDS, int MODE>
+template <int RG, int WORDS, int MODE, bool VAR>
 cudaError_t launch_t(const DecodeArgs& a, size_t smem, cudaStream_t stream) {
-  auto kern = decode_kernel<RG, WORDS, MODE>;
+  auto kern = decode_kernel<RG, WORDS, MODE, VAR>;
   static std::atomic<size_t> raised[kMaxDevices];
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem, raised);
   if (e != cudaSuccess) return e;
@@ -1654,10 +1659,15 @@ cudaError_t launch_t(const DecodeArgs& a, size_t smem, cudaStream_t stream) {
 
 template <int RG, int WORDS>
 cudaError_t launch_mode(const DecodeArgs& a, int mode, size_t smem, cudaStream_t stream) {
+  const bool var = a.meta_f32 || a.gqa_sum || a.simt_bounds;
   switch (mode) {
-    case kModeSelect: return launch_t<RG, WORDS, kModeSelect>(a, smem, stream);
-    case kModeFused: return launch_t<RG, WORDS, kModeFused>(a, smem, stream);
-    case kModeAttend: return launch_t<RG, WORDS, kModeAttend>(a, smem, stream);
+    case kModeSelect:
+      return var ? launch_t<RG, WORDS, kModeSelect, true>(a, smem, stream)
+                 : launch_t<RG, WORDS, kModeSelect, false>(a, smem, stream);
+    case kModeFused:
+      return var ? launch_t<RG, WORDS, kModeFused, true>(a, smem, stream)
+                 : launch_t<RG, WORDS, kModeFused, false>(a, smem, stream);
+    case kModeAttend: return launch_t<RG, WORDS, kModeAttend, false>(a, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }
