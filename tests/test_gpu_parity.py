@@ -371,10 +371,19 @@ def test_host_buffer_step_matches_device_step():
     call = Bnd.prepare("hhr_decode_step_host", d.dims, q_pin, q_dev, d.R, d.W, d.codes, d.meta, d.K,
                        d.V, w.N, d.P, d.k, d.scale, d.page_idx, d.tok_idx, d.n_sel, d.out, out_pin,
                        d.ws, d.ws.numel(), torch.cuda.current_stream().cuda_stream)
-    for _ in range(2):
+    for _ in range(3):   # the first call runs on the stream, the others replay its graph
         call()
         assert np.array_equal(out_pin.numpy(), ref_out)
         assert np.array_equal(_host(d.tok_idx), ref_tok)
+    # a new query in the same pinned buffer: the replay copies what is there now
+    q2 = torch.roll(d.q[0], shifts=1, dims=1).contiguous()
+    hhr.hhr_decode_step(d.dims, q2, d.R, d.W, d.codes, d.meta, d.K, d.V, w.N, d.P, d.k, d.scale,
+                        d.page_idx, d.tok_idx, d.n_sel, d.out, d.ws)
+    ref2 = _host(d.out).copy()
+    assert not np.array_equal(ref2, ref_out)
+    q_pin.copy_(q2.cpu())
+    call()
+    assert np.array_equal(out_pin.numpy(), ref2)
     assert d.status() == hhr.HHR_OK
 
 
