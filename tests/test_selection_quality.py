@@ -8,7 +8,7 @@ Generation", §3.3.1 Fig. 3 and §3.3.2 Fig. 4).  Its R and W are trained;
 here R is a seeded random orthogonal matrix and W a seeded Gaussian, so the
 numbers describe the mechanism on synthetic keys, not the paper's figures.
 R = I turns the page bounds into the raw per-channel min / max of the keys
-(QUEST-style).  The oracle is the judge: it computes the exact top-k keys by
+(QUEST-style).  The oracle decides what the true top-k is: it ranks the keys by
 group logit (max over the group's heads of q_h . k) in double.
 """
 import math
