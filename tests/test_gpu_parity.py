@@ -22,6 +22,8 @@ SMALL = {
     "page64": scaled(get("llama8b_32k"), Hq=8, Hkv=2, N=5000, page=64, P=20, k=300, planted=4),
     "gqa2": scaled(get("llama8b_32k"), Hq=16, Hkv=8, N=3000, P=40, k=200, planted=8),
     "gqa8": scaled(get("llama8b_32k"), Hq=32, Hkv=4, N=3000, P=40, k=200, planted=8),
+    # r = 8 with 256-bit codes: the widest GQA-sum histogram (r b + 1 = 2049 bins)
+    "gqa8_b256": scaled(get("batch8_64k_b256"), B=1, Hq=32, Hkv=4, N=3000, P=40, k=200, planted=8),
 }
 
 _cache = {}
@@ -168,7 +170,7 @@ def variant_state(name, f32):
 
 
 @pytest.mark.parametrize("variant", list(VARIANTS))
-@pytest.mark.parametrize("name", ["llama_20k_ragged", "b256_s32", "gqa8", "page1", "tiny_4k"])
+@pytest.mark.parametrize("name", ["llama_20k_ragged", "b256_s32", "gqa8", "gqa8_b256", "page1", "tiny_4k"])
 def test_variant_matches_oracle(name, variant):
     """HHR_FLAG_META_F32 (float32 page metadata) and HHR_FLAG_GQA_SUM (summed
     group distances) against the oracle's variants: the GPU encode, the
