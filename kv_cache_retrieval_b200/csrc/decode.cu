@@ -798,7 +798,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ D
       // (s * NWARPS + w) * 512: slots [0, kLaneSlots) lie below the R / W
       // buffer, slots [kLaneSlots, kRingSlots) inside it.
       constexpr int PPG = 8;                        // pages per ring group; an A tile is two groups
-      constexpr int G0 = 1;                         // groups in flight while q~ is formed (A/B: 1 beats 0 and 2)
+      constexpr int G0 = 2;                         // groups in flight while q~ is formed (all below R / W)
       constexpr int GR = kRingSlots / PPG;          // groups in flight afterwards
       static_assert(kLaneSlots % PPG == 0 && kRingSlots % PPG == 0 && G0 * PPG <= kLaneSlots,
                     "whole groups per ring; the groups issued before q~ stay below the R / W buffer");
