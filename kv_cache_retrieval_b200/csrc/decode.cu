@@ -32,8 +32,17 @@
 //                      cp.async, online softmax in float32
 //      -- last-arriving CTA merges the C partial softmax states --
 //
+// Variants chosen by hhr_dims.flags (compiled into a second instantiation;
+// with every flag 0 their branches are compiled out): float32 page metadata
+// (phase 1 on the CUDA cores, 1-KiB pages), GQA-sum distances (phase 4 sums
+// over the group's heads; r*b + 1 histogram bins), and phase 1 on the CUDA
+// cores for bf16 metadata (the comparison form of the tensor-core tiles).
+// The attend-only launch also serves dense attention over every valid key
+// (each CTA one contiguous key range, no token list).
+//
 // The kernel is launched as a programmatic dependent of the previous kernel
-// on the stream and waits for it before touching memory.  Inter-CTA waits
+// on the stream; its set-up touches no global memory and may overlap that
+// kernel's tail, and it waits for it before the first global access.  Inter-CTA waits
 // spin on workspace counters with a clock64() limit; on expiry the kernel
 // records HHR_ERR_TIMEOUT and returns.  The last CTA of a unit resets its
 // counter, so the workspace is zero again after each call.
