@@ -20,8 +20,9 @@ import torch
 
 import kv_cache_retrieval_b200 as hhr
 from gpu_harness import QUALITY, bf16_dev
+from kv_cache_retrieval_b200 import fit
 from oracle import oracle as O
-from workloads import get, make_inputs
+from workloads import bf16_bits_to_f32, get, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -34,12 +35,14 @@ def _inp(name):
     return _inputs[name]
 
 
-def _gpu_select(inp, R):
-    """GPU encode with rotation R, then one fused decode step (step 0)."""
+def _gpu_select(inp, R, W=None):
+    """GPU encode with rotation R (and projection W), then one fused decode
+    step (step 0)."""
     w = inp.w
     dims = hhr.make_dims(w.B, w.Hq, w.Hkv, w.d, w.bits, w.page, w.n_cap)
     K, V, q = bf16_dev(inp.K), bf16_dev(inp.V), bf16_dev(inp.q[0])
-    Rt, Wt = torch.from_numpy(np.ascontiguousarray(R)).cuda(), torch.from_numpy(inp.W).cuda()
+    Rt = torch.from_numpy(np.ascontiguousarray(R)).cuda()
+    Wt = torch.from_numpy(np.ascontiguousarray(inp.W if W is None else W)).cuda()
     codes = torch.zeros(w.B, w.Hkv, w.n_cap, w.words, dtype=torch.int32, device="cuda")
     meta = torch.zeros(w.B, w.Hkv, w.np_cap, 2, w.d, dtype=torch.bfloat16, device="cuda")
     hhr.hhr_encode_keys(dims, K, Rt, Wt, 0, w.N, codes, meta)
@@ -85,5 +88,60 @@ def test_recall_of_exact_top_k(name):
         assert 0.0 <= rt <= rp <= 1.0
         res[label] = {"token_recall": round(rt, 4), "page_recall": round(rp, 4),
                       "planted_selected": f"{planted}/{w.units * w.planted}"}
+    QUALITY.append(res)
+    print(res)
+
+
+def _recall(inp, top, page_idx, tok_idx, n_sel):
+    w = inp.w
+    tr, pr = [], []
+    for (b, g), t in top.items():
+        sel = tok_idx[b, g, :n_sel[b, g]]
+        kept = page_idx[b, g][page_idx[b, g] >= 0]
+        tr.append(np.isin(t, sel).mean())
+        pr.append(np.isin(t // w.page, kept).mean())
+    return round(float(np.mean(tr)), 4), round(float(np.mean(pr)), 4)
+
+
+def test_recall_with_fitted_r_and_w():
+    """R and W fitted offline per KV head (kv_cache_retrieval_b200.fit; the
+    paper's §3.3.1 Eqs. 5-9 and §3.3.2 Eqs. 10-15) on 64 seeded training
+    queries, then used by the CUDA path on the workload's own (held-out)
+    query; recall of the exact top-k beside the seeded random R and W."""
+    name = "llama8b_32k"
+    inp = _inp(name)
+    w = inp.w
+    r = w.r
+    units = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+
+    def exact(bg):
+        b, g = bg
+        return O.top_logits(inp.q[0, b, g * r:(g + 1) * r], inp.K[b, g], w.N, w.k)
+
+    with ThreadPoolExecutor(O.default_threads()) as ex:
+        top = dict(zip(units, ex.map(exact, units)))
+    gen = torch.Generator(device="cuda").manual_seed(0x48485201)
+    R_fit = np.empty_like(inp.R)
+    W_fit = np.empty_like(inp.W)
+    losses = []
+    for g in range(w.Hkv):
+        K = torch.from_numpy(bf16_bits_to_f32(inp.K[0, g, :w.N])).cuda()
+        Q = torch.randn(64, w.d, device="cuda", generator=gen).to(torch.bfloat16).float()
+        W0 = torch.from_numpy(inp.W[g]).cuda() / math.sqrt(w.d)
+        R, hr = fit.fit_rotation(K, Q, W0, w.page, keep=w.P, top_k=w.k, steps=150)
+        W, hw = fit.fit_projection(K, Q, R, W0, w.page, keep=w.P, top_n=w.k, steps=150)
+        assert torch.allclose(R.T @ R, torch.eye(w.d, device="cuda"), atol=1e-4)
+        R_fit[g], W_fit[g] = R.cpu().numpy(), W.cpu().numpy()
+        losses.append((round(hr[0], 4), round(min(hr), 4), round(hw[0], 4), round(min(hw), 4)))
+    res = {"workload": name, "k": w.k, "P": w.P,
+           "fit objective (R start/best, W start/best), head 0": losses[0]}
+    for label, R, W in (("random R, W", inp.R, inp.W), ("fitted R, W", R_fit, W_fit),
+                        ("fitted R, random W", R_fit, inp.W)):
+        page_idx, tok_idx, n_sel = _gpu_select(inp, R, W)
+        tr, pr = _recall(inp, top, page_idx, tok_idx, n_sel)
+        assert 0.0 <= tr <= pr <= 1.0
+        res[label] = {"token_recall": tr, "page_recall": pr}
+    for (r0, r1, w0, w1) in losses:
+        assert r1 <= r0 and w1 <= w0
     QUALITY.append(res)
     print(res)
