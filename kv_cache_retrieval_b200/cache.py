@@ -15,8 +15,10 @@ from . import _binding as B
 
 class HHRCache:
     def __init__(self, *, batch, q_heads, kv_heads, capacity, bits=128, page=16, head_dim=128,
-                 P=512, k=4096, device="cuda"):
-        self.dims = B.make_dims(batch, q_heads, kv_heads, head_dim, bits, page, capacity)
+                 P=512, k=4096, device="cuda", flags=0):
+        """flags: HHR_FLAG_META_F32 (float32 page metadata) and / or
+        HHR_FLAG_GQA_SUM (summed group distances); 0 for the defaults."""
+        self.dims = B.make_dims(batch, q_heads, kv_heads, head_dim, bits, page, capacity, flags)
         self.device = torch.device(device)
         self.P, self.k = P, k
         n_pages = (capacity + page - 1) // page
@@ -24,7 +26,8 @@ class HHRCache:
         self.K = torch.zeros(batch, kv_heads, capacity, head_dim, dtype=torch.bfloat16, device=dev)
         self.V = torch.zeros_like(self.K)
         self.codes = torch.zeros(batch, kv_heads, capacity, bits // 32, dtype=torch.int32, device=dev)
-        self.meta = torch.zeros(batch, kv_heads, n_pages, 2, head_dim, dtype=torch.bfloat16, device=dev)
+        meta_dtype = torch.float32 if flags & B.HHR_FLAG_META_F32 else torch.bfloat16
+        self.meta = torch.zeros(batch, kv_heads, n_pages, 2, head_dim, dtype=meta_dtype, device=dev)
         self.R = torch.zeros(kv_heads, head_dim, head_dim, dtype=torch.float32, device=dev)
         self.W = torch.zeros(kv_heads, head_dim, bits, dtype=torch.float32, device=dev)
         self.page_idx = torch.empty(batch, kv_heads, P, dtype=torch.int32, device=dev)
@@ -59,6 +62,13 @@ class HHRCache:
                           n_valid, self.P, self.k, self.scale, self.page_idx, self.tok_idx,
                           self.n_sel, self.out, self.workspace, None, stream)
         return self.out
+
+    def dense_attend(self, q, n_valid, out=None, stream=None):
+        """Dense attention over every valid key (the comparator of the sparse
+        step)."""
+        B.hhr_dense_attend(self.dims, q, self.K, self.V, n_valid, self.scale,
+                           self.out if out is None else out, self.workspace, None, stream)
+        return self.out if out is None else out
 
     def status(self, stream=None) -> int:
         return B.hhr_read_status(self.workspace, stream)

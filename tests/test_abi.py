@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import kv_cache_retrieval_b200 as hhr
 from kv_cache_retrieval_b200 import _binding as Bnd
@@ -160,3 +161,14 @@ def test_variant_flags_validation():
     plain, summed = _dims(), _dims(flags=hhr.HHR_FLAG_GQA_SUM)
     assert hhr.hhr_workspace_size(summed, 64, 256) > hhr.hhr_workspace_size(plain, 64, 256)
     assert hhr.hhr_workspace_size(_dims(flags=16), 64, 256) == 0
+
+
+def test_cache_buffers_follow_the_flags():
+    """HHRCache sizes its buffers from the dims (host-side, no kernel runs)."""
+    base = dict(batch=1, q_heads=8, kv_heads=2, capacity=512, P=8, k=32, device="cpu")
+    c0 = hhr.HHRCache(**base)
+    c1 = hhr.HHRCache(**base, flags=hhr.HHR_FLAG_META_F32 | hhr.HHR_FLAG_GQA_SUM)
+    assert c0.meta.dtype == torch.bfloat16 and c1.meta.dtype == torch.float32
+    assert c1.meta.shape == c0.meta.shape == (1, 2, 32, 2, 128)
+    assert c1.workspace.numel() > c0.workspace.numel()   # wider distance histograms
+    assert c1.dims.flags == hhr.HHR_FLAG_META_F32 | hhr.HHR_FLAG_GQA_SUM
