@@ -170,8 +170,8 @@ size_t hhr_workspace_size(const hhr_dims* dims, int32_t P, int32_t k);
  * Retrieval for one decode step (GKR then LHP) for every (sequence, KV head):
  * query rotation and codes, page bounds of the ceil(n_valid/page) pages
  * (Eq. 3, max over the group), the P best pages, Hamming distances of every
- * valid token of those pages (Eq. 2, min over the group), and the k closest
- * tokens.
+ * valid token of those pages (Eq. 2, min over the group; the sum with
+ * HHR_FLAG_GQA_SUM), and the k closest tokens.
  *   q        device, read:  bf16 [B][Hq][d].
  *   R, W     device, read:  as for hhr_encode_keys.
  *   codes, meta device, read: encoded keys [0, n_valid).
@@ -181,7 +181,7 @@ size_t hhr_workspace_size(const hhr_dims* dims, int32_t P, int32_t k);
  *   page_idx, tok_idx, n_sel device, write (layouts above).
  *   dbg_U    device, write, nullable: f32 [B][Hkv][ceil(n_valid/page)] group
  *            page bounds.
- *   dbg_D    device, write, nullable: i32 [B][Hkv][P*page] distance of token
+ *   dbg_D    device, write, nullable: i32 [B][Hkv][P*page] group distance of token
  *            page_idx[slot]*page + t at [slot*page + t]; -1 for empty slots and
  *            tokens >= n_valid.
  *   workspace device, read+write: at least hhr_workspace_size(dims, P, k) bytes.
